@@ -1,0 +1,34 @@
+"""CPU oracle for the fused W4 + sparse-residual linear (test infrastructure).
+
+A plain, slow, fp64 restatement of what the hot path computes, written from
+the MosaicQuant pages:
+
+  * decompose.py - inlier-outlier disaggregation W ~= Q(W) + R: a dense 4-bit
+    base and a sparse 4-bit residual that patches the worst-quantized entries
+    (MosaicQuant, "Methodology", 1. Inlier-Outlier Disaggregation, the
+    equation W_hat ~= Q(W_hat) + R; both parts 4-bit).
+  * pack.py      - the device byte layout of that decomposition, and unpack.
+  * linear.py    - the product Y = X * W_hat^T, W_hat = deq(Q) + R, as dense
+    base plus a CSR loop (the "reduction-add" of ZipperEngine's pipeline) and
+    as a brute-force triple loop.
+  * tolerance.py - the parity metrics used to accept a bf16 GPU output.
+
+This package is test infrastructure. Only tests/, __graft_entry__.smoke() and
+bench.py's CPU-baseline / reference arm may import it. The product path
+(bit_gemm_w4_b200) never imports it, and it imports nothing from the product.
+Every function is pinned by CPU tests against brute force, closed forms or
+library routines (tests/test_oracle_*.py); none is "parity unpinned".
+"""
+
+from .decompose import (Decomposition, decompose, from_arrays, fp16_rne,
+                        residual_count, quantize_base, select_residual,
+                        quantize_residual)
+from .pack import pack, unpack
+from .linear import dequant_base, w_hat, linear, linear_brute
+from .tolerance import parity_report
+
+__all__ = [
+    "Decomposition", "decompose", "from_arrays", "fp16_rne", "residual_count",
+    "quantize_base", "select_residual", "quantize_residual", "pack", "unpack",
+    "dequant_base", "w_hat", "linear", "linear_brute", "parity_report",
+]
