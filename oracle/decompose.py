@@ -116,7 +116,9 @@ def quantize_base(W: np.ndarray, group: int):
     s = np.where(hi == lo, np.float16(1.0), s)
     s = np.where((s == 0) & (hi > lo), np.float16(2.0 ** -24), s)
     s64 = s.astype(np.float64)
-    z = np.clip(np.rint(-lo / s64), 0.0, 15.0)
+    # z is an integer code 0..15; "+ 0.0" keeps its fp16 encoding canonical
+    # (+0, not the -0 that -lo/s gives when lo = 0)
+    z = np.clip(np.rint(-lo / s64), 0.0, 15.0) + 0.0
     q = np.clip(np.rint(v / s64[..., None]) + z[..., None], 0.0, 15.0)
     deq = (q - z[..., None]) * s64[..., None]
     return (q.astype(np.uint8).reshape(N, K), s.astype(np.float16),

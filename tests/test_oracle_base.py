@@ -116,3 +116,9 @@ def test_hand_derived_example(golden):
     np.testing.assert_array_equal(d.q[0], [int(x) for x in f["q"]])
     assert d.s.view(np.uint16)[0, 0] == int(f["s_bits"][0], 16)
     assert d.z.view(np.uint16)[0, 0] == int(f["z_bits"][0], 16)
+
+
+def test_zero_point_encoding_is_canonical():
+    W = np.abs(np.random.default_rng(4).standard_normal((1, 128))).astype(np.float32)
+    q, s, z, deq = quantize_base(W, 128)
+    assert z.view(np.uint16)[0, 0] == 0x0000      # +0, never -0
