@@ -1,0 +1,454 @@
+"""Benchmark of the fused W4 + sparse-residual linear on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the hot path over one batch: the 7B-shaped decode
+workload (one token through q/k/v/o 4096x4096, gate/up 11008x4096 and down
+4096x11008 linears, rho = 0.5 %), i.e. three fused launches. The metric is
+the decode HBM throughput in TB/s of algorithmic bytes (each packed array, X
+and Y once). Weights rotate through enough independent packed copies that
+every step reads them from HBM, not L2.
+
+Every rank (one per GPU under torchrun) runs the same workload on its own GPU
+(independent replicas, weak scaling): the layer has no exchange step, so there
+is no data-path collective. Rank 0 prints one JSON line.
+
+Also reported (secondary): the 70B-MLP batched decode (M = 16) in TB/s and
+the prefill (M = 2048) in TFLOP/s, each with its roofline fraction.
+
+--impl reference times the fp64 CPU oracle on a bounded row sample of the
+same workload (rank 0 only) and prints the same JSON line with
+"impl": "reference".
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused W4+residual linear: decode HBM TB/s, prefill TFLOP/s, % of roofline"
+WORKLOAD = ("7B-shaped decode, M=1: q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008; "
+            "int4 g128 base + 0.5% int4 CSR residual; bf16 X with 4 channels x20")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def alg_bytes(M: int, N: int, K: int, nnz: int) -> int:
+    """Algorithmic bytes of one product: packed base, scale/zero words, CSR
+    (row_ptr, col, val, rscale), X and Y, each once."""
+    return (N * K // 2 + 4 * N * (K // 128) + 4 * (N + 1) + 2 * nnz + (nnz + 1) // 2 + 2 * N
+            + 2 * M * K + 2 * M * N)
+
+
+def alg_flops(M: int, N: int, K: int, nnz: int) -> int:
+    return 2 * M * N * K + 2 * M * nnz
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU is loaded."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+class DecodeSet:
+    """Packed copies of one workload's shapes plus device X / Y buffers."""
+
+    def __init__(self, mq, torch, name: str, copies: int, dev):
+        from bit_gemm_w4_b200 import synth
+        cfg = synth.WORKLOADS[name]
+        self.M = cfg["M"]
+        self.shapes = cfg["shapes"]
+        self.weights = []     # [copy][shape]
+        self.nnz = []
+        for c in range(copies):
+            row = []
+            for i, (N, K) in enumerate(self.shapes):
+                W = synth.weight(N, K, std=cfg["w_std"], outlier_frac=cfg["w_outlier_frac"],
+                                 outlier_cols=cfg["w_outlier_cols"], seed=1000 * (i + 1) + 17 * c)
+                w = mq.Weight.pack(W, cfg["rho"])
+                row.append(w)
+                if c == 0:
+                    self.nnz.append(w.info()["nnz"])
+                del W
+            self.weights.append(row)
+        self.X = []
+        self.Y = []
+        for i, (N, K) in enumerate(self.shapes):
+            X = synth.activations(self.M, K, seed=7 + i, channels=cfg["x_channels"],
+                                  mult=cfg["x_mult"])
+            self.X.append(X.to(dev))
+            self.Y.append(torch.empty((self.M, N), dtype=torch.bfloat16, device=dev))
+        self.bytes_per_launch = [alg_bytes(self.M, N, K, nz)
+                                 for (N, K), nz in zip(self.shapes, self.nnz)]
+        self.flops_per_launch = [alg_flops(self.M, N, K, nz)
+                                 for (N, K), nz in zip(self.shapes, self.nnz)]
+
+    def launch(self, copy: int, i: int, stream):
+        w = self.weights[copy][i]
+        w.linear_raw(self.X[i].data_ptr(), self.M, self.Y[i].data_ptr(), stream=stream)
+
+
+def time_graph_steps(torch, ds: DecodeSet, steps: int, warmup: int, stream, chunk: int,
+                     dist_ctx, sampler_gpu: int):
+    """Capture `chunk` steps (rotating copies) with external timing events
+    around each launch, replay to cover exactly `steps` steps. Returns total
+    ms (max over ranks), per-launch ms of the last chunk, clocks."""
+    copies = len(ds.weights)
+    nsh = len(ds.shapes)
+    for s in range(warmup):
+        for i in range(nsh):
+            ds.launch(s % copies, i, stream)
+    torch.cuda.synchronize()
+
+    def capture(nsteps):
+        evs = [torch.cuda.Event(enable_timing=True, external=True)
+               for _ in range(nsteps * nsh + 1)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            evs[0].record(stream)
+            for s in range(nsteps):
+                for i in range(nsh):
+                    ds.launch(s % copies, i, stream)
+                    evs[s * nsh + i + 1].record(stream)
+        return g, evs
+
+    full, rem = divmod(steps, chunk)
+    g, evs = capture(chunk) if full else (None, None)
+    g_rem, evs_rem = capture(rem) if rem else (None, None)
+    # settle clocks under the same load before the timed region
+    t_end = time.time() + 0.5
+    with ClockSampler(sampler_gpu) as clk:
+        while time.time() < t_end:
+            (g or g_rem).replay()
+        torch.cuda.synchronize()
+        dist_ctx.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(full):
+            g.replay()
+        if rem:
+            g_rem.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dist_ctx.barrier()
+    ms = dist_ctx.max(e0.elapsed_time(e1))
+    last_evs = evs if evs is not None else evs_rem
+    per = [last_evs[j].elapsed_time(last_evs[j + 1]) for j in range(len(last_evs) - 1)]
+    per_shape = [statistics.mean(per[i::nsh]) for i in range(nsh)]
+    return ms, per_shape, clk.summary()
+
+
+def time_e2e(torch, ds: DecodeSet, steps: int, stream, dist_ctx):
+    """The public API with host buffers: per step H2D of X from pinned memory,
+    the fused calls, D2H of Y into pinned memory."""
+    copies = len(ds.weights)
+    hx = [x.cpu().pin_memory() for x in ds.X]
+    hy = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in ds.Y]
+    h2d = sum(x.numel() * 2 for x in hx)
+    d2h = sum(y.numel() * 2 for y in hy)
+
+    def step(s):
+        for i in range(len(ds.shapes)):
+            ds.X[i].copy_(hx[i], non_blocking=True)
+            ds.launch(s % copies, i, stream)
+            hy[i].copy_(ds.Y[i], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for s in range(3):
+            step(s)
+        torch.cuda.synchronize()
+        dist_ctx.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(steps):
+            step(s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dist_ctx.barrier()
+    return dist_ctx.max(e0.elapsed_time(e1)), h2d, d2h
+
+
+class DistCtx:
+    def __init__(self, torch):
+        self.torch = torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        t = self.torch.tensor([v], dtype=self.torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def secondary(torch, mq, dev, stream, pk, which: str, reps: int):
+    """One secondary workload: device time per launch over `reps` launches."""
+    from bit_gemm_w4_b200 import synth
+    ds = DecodeSet(mq, torch, which, 1, dev)
+    N, K = ds.shapes[0]
+    for _ in range(3):
+        ds.launch(0, 0, stream)
+    torch.cuda.synchronize()
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    times = []
+    for _ in range(reps):
+        flush.zero_()                      # evict L2 between launches
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ds.launch(0, 0, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    by, fl = ds.bytes_per_launch[0], ds.flops_per_launch[0]
+    out = {"workload": which, "M": ds.M, "N": N, "K": K, "nnz": ds.nnz[0], "ms": ms,
+           "TB_s": by / ms / 1e9, "TFLOP_s": fl / ms / 1e9}
+    if which == "prefill":
+        peak = pk["bf16_tflops"]
+        out["roofline"] = {"bound": "tensor", "achieved": fl / ms / 1e9, "peak": peak,
+                           "unit": "TFLOP/s", "frac": fl / ms / 1e9 / peak}
+    else:
+        peak = pk["hbm_gbs"]
+        out["roofline"] = {"bound": "hbm", "achieved": by / ms / 1e6, "peak": peak,
+                           "unit": "GB/s", "frac": by / ms / 1e6 / peak}
+    del ds
+    return out
+
+
+def run_ours(args):
+    import torch
+    from bit_gemm_w4_b200 import mosaicq as mq
+    dist_ctx = DistCtx(torch)
+    dev = torch.device("cuda", dist_ctx.local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    pk, pk_src = peaks()
+    # enough copies that consecutive reuse of one copy is > 2x L2 apart
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per_copy = sum(alg_bytes(1, N, K, 0) for N, K in [(4096, 4096), (11008, 4096), (4096, 11008)])
+    copies = max(2, int(np.ceil(2.0 * l2 / per_copy)) + 1)
+    ds = DecodeSet(mq, torch, "7b_decode", copies, dev)
+    chunk = min(args.steps, 100)
+    ms, per_shape, clocks = time_graph_steps(torch, ds, args.steps, args.warmup, stream, chunk,
+                                             dist_ctx, dist_ctx.local)
+    step_bytes = sum(ds.bytes_per_launch)
+    value = step_bytes * args.steps * dist_ctx.world / (ms * 1e-3) / 1e12
+    e2e_steps = min(args.steps, 500)
+    ms_e2e, h2d, d2h = time_e2e(torch, ds, e2e_steps, stream, dist_ctx)
+    e2e = step_bytes * e2e_steps * dist_ctx.world / (ms_e2e * 1e-3) / 1e12
+    # dominant kernel: the fused decode kernel (all three launches of a step)
+    kern_ms = sum(per_shape)
+    achieved = step_bytes / (kern_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC, "value": round(value, 4), "unit": "TB/s", "n_gpus": dist_ctx.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; no model weights)",
+        "config": {"workload": WORKLOAD, "M": 1,
+                   "shapes_NxK": [list(s) for s in ds.shapes], "rho": 0.005,
+                   "alg_bytes_per_step": step_bytes,
+                   "l2": f"inputs larger than L2: {copies} rotating weight copies "
+                         f"({copies * step_bytes / 1e6:.0f} MB) vs L2 {l2 / 1e6:.0f} MB",
+                   "parallelism": f"replicas x{dist_ctx.world}", "timing": "CUDA graph replay"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                     "peak_source": pk_src,
+                     "per_launch_us": {f"{N}x{K}": round(t * 1e3, 3)
+                                       for (N, K), t in zip(ds.shapes, per_shape)}},
+        "e2e": {"value": round(e2e, 4), "unit": "TB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps * len(ds.shapes),
+        "clocks": clocks,
+    }
+    del ds
+    torch.cuda.empty_cache()
+    if not args.no_secondary:
+        sec = []
+        for which in ("70b_mlp", "prefill"):
+            try:
+                sec.append(secondary(torch, mq, dev, stream, pk, which, reps=10))
+            except Exception as e:  # report, never hide
+                sec.append({"workload": which, "error": str(e)})
+            torch.cuda.empty_cache()
+        result["secondary"] = sec
+    if dist_ctx.rank == 0 and not args.skip_cpu_baseline and dist_ctx.world == 1:
+        result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+    if dist_ctx.rank == 0:
+        print(json.dumps(result), flush=True)
+    dist_ctx.close()
+
+
+# ------------------------------------------------------------------ oracle arm
+def _oracle_sample(rows_per_shape: int):
+    """Row samples of the 7B decode workload decomposed by the oracle."""
+    import oracle
+    from bit_gemm_w4_b200 import synth
+    cfg = synth.WORKLOADS["7b_decode"]
+    parts = []
+    for i, (N, K) in enumerate(cfg["shapes"]):
+        rows = np.linspace(0, N - 1, rows_per_shape).astype(np.int64)
+        W, X, rho = synth.workload_inputs("7b_decode", i, rows=rows)
+        d = oracle.decompose(W, rho)
+        parts.append((X, d, alg_bytes(1, rows_per_shape, K, d.nnz)))
+    return parts
+
+
+def cpu_baseline(budget_s: float = 10.0, rows_per_shape: int = 512):
+    import oracle
+    parts = _oracle_sample(rows_per_shape)
+    byts = sum(p[2] for p in parts)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        for X, d, _ in parts:
+            oracle.linear(X, d)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": byts * n / dt / 1e12, "unit": "TB/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"{rows_per_shape} rows of each of the 3 shapes (M=1), {n} passes in {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    rows = 64
+    parts = _oracle_sample(rows)
+    byts = sum(p[2] for p in parts)
+    for _ in range(args.warmup):
+        for X, d, _ in parts:
+            oracle.linear(X, d)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for X, d, _ in parts:
+            oracle.linear(X, d)
+    dt = time.perf_counter() - t0
+    value = byts * args.steps / dt / 1e12
+    cores = len(os.sched_getaffinity(0))
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; no model weights)",
+        "config": {"workload": WORKLOAD, "M": 1, "sample": f"{rows} rows of each shape"},
+        "cpu_baseline": {"value": value, "unit": "TB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} rows of each of the 3 shapes per step"},
+        "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,375 @@
+// C ABI of libmosaicq (include/mosaicq.h): validation, packing + upload,
+// TMA descriptors, kernel dispatch, export and error reporting.
+//
+// MosaicQuant (gist.science/paper/2606.15652): "Methodology" 1. defines the
+// 4-bit disaggregated weight W ~= Q(W) + R built once by mq_pack;
+// "Methodology" 3. (ZipperEngine) defines the fused product mq_linear runs.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+#include "kernels.h"
+
+struct mq_weight {
+    int device = -1;
+    mq::DeviceWeight d{};
+    int64_t max_row_nnz = 0;
+    int64_t device_bytes = 0;
+    std::vector<void *> allocations;
+    std::vector<int32_t> host_row_ptr;  // for residual tile statistics
+    mutable std::mutex maps_mu;
+    mutable std::vector<mq::MapSet *> maps;
+    ~mq_weight() {
+        for (auto *m : maps) delete m;
+    }
+};
+
+namespace mq {
+
+namespace {
+thread_local std::string g_last_error;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool encode_2d_u32(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                   uint32_t box_inner, uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 4};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+mq_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(e == cudaErrorMemoryAllocation ? MQ_ERR_OUT_OF_MEMORY : MQ_ERR_CUDA,
+                std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+template <class T>
+mq_status upload(mq_weight *w, T **dst, const T *src, size_t count, size_t pad_bytes,
+                 cudaStream_t stream) {
+    size_t bytes = count * sizeof(T) + pad_bytes;
+    void *p = nullptr;
+    cudaError_t e = cudaMalloc(&p, bytes > 0 ? bytes : 16);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc");
+    w->allocations.push_back(p);
+    w->device_bytes += static_cast<int64_t>(bytes);
+    if (pad_bytes) {
+        e = cudaMemsetAsync(p, 0, bytes, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    }
+    if (count) {
+        e = cudaMemcpyAsync(p, src, count * sizeof(T), cudaMemcpyHostToDevice, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync");
+    }
+    *dst = static_cast<T *>(p);
+    return MQ_OK;
+}
+
+mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **out) {
+    *out = nullptr;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "no usable CUDA device");
+    mq_weight *w = new (std::nothrow) mq_weight();
+    if (!w) return fail(MQ_ERR_OUT_OF_MEMORY, "host allocation failed");
+    w->device = dev;
+    DeviceWeight &d = w->d;
+    d.N = hp.N;
+    d.K = hp.K;
+    d.G = hp.G;
+    d.Gp = hp.Gp;
+    d.nnz = hp.nnz;
+    mq_status st = MQ_OK;
+    uint32_t *qw = nullptr, *sz = nullptr;
+    int32_t *rp = nullptr;
+    uint16_t *col = nullptr, *rs = nullptr;
+    uint8_t *val = nullptr;
+    int *err = nullptr;
+    int zero = 0;
+    if (!st) st = upload(w, &qw, hp.qweight.data(), hp.qweight.size(), 0, stream);
+    if (!st) st = upload(w, &sz, hp.sz.data(), hp.sz.size(), 0, stream);
+    if (!st) st = upload(w, &rp, hp.row_ptr.data(), hp.row_ptr.size(), 0, stream);
+    if (!st) st = upload(w, &col, hp.col.data(), hp.col.size(), 64, stream);
+    if (!st) st = upload(w, &val, hp.val.data(), hp.val.size(), 64, stream);
+    if (!st) st = upload(w, &rs, hp.rscale.data(), hp.rscale.size(), 0, stream);
+    if (!st) st = upload(w, &err, &zero, 1, 0, stream);
+    if (!st) {
+        e = cudaStreamSynchronize(stream);
+        if (e != cudaSuccess) st = cuda_fail(e, "upload");
+    }
+    if (st) {
+        mq_free(w);
+        return st;
+    }
+    d.qweight = qw;
+    d.sz = sz;
+    d.row_ptr = rp;
+    d.col = col;
+    d.val = val;
+    d.rscale = rs;
+    d.err = err;
+    w->host_row_ptr = hp.row_ptr;
+    for (int64_t n = 0; n < hp.N; ++n)
+        w->max_row_nnz = std::max<int64_t>(w->max_row_nnz, hp.row_ptr[n + 1] - hp.row_ptr[n]);
+    *out = w;
+    return MQ_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+void set_error(const std::string &msg) { g_last_error = msg; }
+
+mq_status fail(mq_status s, const std::string &msg) {
+    g_last_error = msg;
+    return s;
+}
+
+const DeviceWeight &weight_device(const mq_weight *w) { return w->d; }
+
+const MapSet *weight_maps(const mq_weight *w, int bn, int gs) {
+    std::lock_guard<std::mutex> lock(w->maps_mu);
+    for (auto *m : w->maps)
+        if (m->bn == bn && m->gs == gs) return m;
+    MapSet *m = new (std::nothrow) MapSet();
+    if (!m) return nullptr;
+    m->bn = bn;
+    m->gs = gs;
+    const DeviceWeight &d = w->d;
+    if (!encode_2d_u32(&m->w, d.qweight, d.K / 8, d.N, 16, bn) ||
+        !encode_2d_u32(&m->sz, d.sz, d.Gp, d.N, gs, bn)) {
+        delete m;
+        fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+        return nullptr;
+    }
+    for (int64_t r = 0; r < d.N; r += bn) {
+        int64_t r1 = std::min<int64_t>(d.N, r + bn);
+        m->max_tile_nnz = std::max<int64_t>(m->max_tile_nnz,
+                                            w->host_row_ptr[r1] - w->host_row_ptr[r]);
+    }
+    w->maps.push_back(m);
+    return m;
+}
+
+}  // namespace mq
+
+using namespace mq;
+
+extern "C" {
+
+const char *mq_strerror(mq_status s) {
+    switch (s) {
+        case MQ_OK: return "ok";
+        case MQ_ERR_INVALID_ARG: return "invalid argument";
+        case MQ_ERR_UNSUPPORTED: return "unsupported";
+        case MQ_ERR_OUT_OF_MEMORY: return "out of memory";
+        case MQ_ERR_CUDA: return "CUDA error";
+        case MQ_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+const char *mq_last_error(void) { return g_last_error.c_str(); }
+
+mq_status mq_residual_nnz(int64_t N, int64_t K, const mq_pack_opts *opts, int64_t *nnz) {
+    if (!nnz) return fail(MQ_ERR_INVALID_ARG, "nnz is NULL");
+    if (mq_status st = check_shape(N, K, opts)) return st;
+    *nnz = N * residual_count(K, opts->residual_density);
+    return MQ_OK;
+}
+
+mq_status mq_pack_host(const float *W_host, int64_t N, int64_t K, const mq_pack_opts *opts,
+                       mq_host_packed *out) {
+    if (!W_host || !out) return fail(MQ_ERR_INVALID_ARG, "NULL pointer");
+    if (mq_status st = check_shape(N, K, opts)) return st;
+    if (!out->qweight || !out->sz || !out->row_ptr || !out->rscale)
+        return fail(MQ_ERR_INVALID_ARG, "an output buffer is NULL");
+    HostDecomp d;
+    if (mq_status st = decompose_host(W_host, N, K, opts->residual_density, d)) return st;
+    if (!d.col.empty() && (!out->col || !out->val))
+        return fail(MQ_ERR_INVALID_ARG, "col/val buffers are NULL");
+    HostPacked p;
+    pack_host(view_of(d), p);
+    std::memcpy(out->qweight, p.qweight.data(), p.qweight.size() * 4);
+    for (int64_t n = 0; n < N; ++n)
+        std::memcpy(out->sz + n * p.G, p.sz.data() + n * p.Gp, p.G * 4);
+    std::memcpy(out->row_ptr, p.row_ptr.data(), p.row_ptr.size() * 4);
+    if (p.nnz) {
+        std::memcpy(out->col, p.col.data(), p.col.size() * 2);
+        std::memcpy(out->val, p.val.data(), p.val.size());
+    }
+    std::memcpy(out->rscale, p.rscale.data(), p.rscale.size() * 2);
+    return MQ_OK;
+}
+
+mq_status mq_pack(const float *W_host, int64_t N, int64_t K, const mq_pack_opts *opts,
+                  mq_stream stream, mq_weight **out) {
+    if (!out) return fail(MQ_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (!W_host) return fail(MQ_ERR_INVALID_ARG, "W is NULL");
+    if (mq_status st = check_shape(N, K, opts)) return st;
+    HostDecomp d;
+    if (mq_status st = decompose_host(W_host, N, K, opts->residual_density, d)) return st;
+    HostPacked p;
+    try {
+        pack_host(view_of(d), p);
+    } catch (const std::bad_alloc &) {
+        return fail(MQ_ERR_OUT_OF_MEMORY, "host allocation for packing failed");
+    }
+    return upload_packed(p, reinterpret_cast<cudaStream_t>(stream), out);
+}
+
+mq_status mq_pack_decomposed(const mq_decomp *dec, mq_stream stream, mq_weight **out) {
+    if (!out) return fail(MQ_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (mq_status st = validate_decomp(dec)) return st;
+    HostPacked p;
+    try {
+        pack_host(*dec, p);
+    } catch (const std::bad_alloc &) {
+        return fail(MQ_ERR_OUT_OF_MEMORY, "host allocation for packing failed");
+    }
+    return upload_packed(p, reinterpret_cast<cudaStream_t>(stream), out);
+}
+
+void mq_free(mq_weight *w) {
+    if (!w) return;
+    int prev = -1;
+    bool switched = false;
+    if (w->device >= 0 && cudaGetDevice(&prev) == cudaSuccess && prev != w->device)
+        switched = cudaSetDevice(w->device) == cudaSuccess;
+    for (void *p : w->allocations) cudaFree(p);
+    if (switched) cudaSetDevice(prev);
+    delete w;
+}
+
+mq_status mq_get_info(const mq_weight *w, mq_info *out) {
+    if (!w || !out) return fail(MQ_ERR_INVALID_ARG, "NULL pointer");
+    out->N = w->d.N;
+    out->K = w->d.K;
+    out->nnz = w->d.nnz;
+    out->group_size = kGroup;
+    out->device = w->device;
+    out->device_bytes = w->device_bytes;
+    out->max_row_nnz = w->max_row_nnz;
+    return MQ_OK;
+}
+
+mq_status mq_export(const mq_weight *w, mq_host_packed *out) {
+    if (!w || !out) return fail(MQ_ERR_INVALID_ARG, "NULL pointer");
+    if (!out->qweight || !out->sz || !out->row_ptr || !out->rscale ||
+        (w->d.nnz && (!out->col || !out->val)))
+        return fail(MQ_ERR_INVALID_ARG, "an output buffer is NULL");
+    int prev = -1;
+    if (cudaGetDevice(&prev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
+    if (prev != w->device && cudaSetDevice(w->device) != cudaSuccess)
+        return fail(MQ_ERR_CUDA, "cudaSetDevice failed");
+    const DeviceWeight &d = w->d;
+    cudaError_t e = cudaDeviceSynchronize();
+    auto cp = [&](void *dst, const void *src, size_t bytes) {
+        if (e == cudaSuccess && bytes) e = cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost);
+    };
+    cp(out->qweight, d.qweight, size_t(d.N) * d.K / 8 * 4);
+    if (e == cudaSuccess)
+        e = cudaMemcpy2D(out->sz, d.G * 4, d.sz, d.Gp * 4, d.G * 4, d.N, cudaMemcpyDeviceToHost);
+    cp(out->row_ptr, d.row_ptr, size_t(d.N + 1) * 4);
+    cp(out->col, d.col, size_t(d.nnz) * 2);
+    cp(out->val, d.val, size_t(d.nnz + 1) / 2);
+    cp(out->rscale, d.rscale, size_t(d.N) * 2);
+    if (prev != w->device) cudaSetDevice(prev);
+    if (e != cudaSuccess) return cuda_fail(e, "mq_export");
+    return MQ_OK;
+}
+
+mq_status mq_device_error(const mq_weight *w, mq_stream stream, int32_t *code) {
+    if (!w || !code) return fail(MQ_ERR_INVALID_ARG, "NULL pointer");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    int v = 0;
+    if (e == cudaSuccess) e = cudaMemcpy(&v, w->d.err, 4, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && v) e = cudaMemset(w->d.err, 0, 4);
+    if (e != cudaSuccess) return cuda_fail(e, "mq_device_error");
+    *code = v;
+    return v ? fail(MQ_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait") : MQ_OK;
+}
+
+mq_status mq_linear_path(const mq_weight *w, const void *X, int64_t M, void *Y, mq_stream stream,
+                         mq_path path) {
+    if (!w) return fail(MQ_ERR_INVALID_ARG, "weight handle is NULL");
+    if (M < 0) return fail(MQ_ERR_INVALID_ARG, "M must be >= 0");
+    if (M == 0) return MQ_OK;
+    if (!X || !Y) return fail(MQ_ERR_INVALID_ARG, "X or Y is NULL");
+    if (!aligned16(X) || !aligned16(Y)) return fail(MQ_ERR_INVALID_ARG, "X and Y must be 16-byte aligned");
+    if (M > (int64_t(1) << 31) - 1) return fail(MQ_ERR_INVALID_ARG, "M too large");
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
+    if (dev != w->device)
+        return fail(MQ_ERR_INVALID_ARG, "the current device is not the device that packed the weight");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (path == MQ_PATH_AUTO) path = (M <= 16) ? MQ_PATH_DECODE : MQ_PATH_PREFILL;
+    switch (path) {
+        case MQ_PATH_DECODE:
+            if (M > 16) return fail(MQ_ERR_UNSUPPORTED, "the decode kernel serves M <= 16");
+            return launch_decode(w, X, static_cast<int>(M), Y, s);
+        case MQ_PATH_PREFILL:
+            return launch_prefill(w, X, M, Y, s);
+        default:
+            return fail(MQ_ERR_INVALID_ARG, "unknown path");
+    }
+}
+
+mq_status mq_linear_unfused(const mq_weight *w, const void *X, int64_t M, void *Y,
+                            void *workspace, size_t workspace_bytes, mq_stream stream) {
+    if (!w) return fail(MQ_ERR_INVALID_ARG, "weight handle is NULL");
+    if (M < 0) return fail(MQ_ERR_INVALID_ARG, "M must be >= 0");
+    if (M == 0) return MQ_OK;
+    if (!X || !Y || !workspace) return fail(MQ_ERR_INVALID_ARG, "X, Y or workspace is NULL");
+    if (!aligned16(X) || !aligned16(Y) || !aligned16(workspace))
+        return fail(MQ_ERR_INVALID_ARG, "X, Y and workspace must be 16-byte aligned");
+    if (M > (int64_t(1) << 31) - 1) return fail(MQ_ERR_INVALID_ARG, "M too large");
+    if (workspace_bytes < static_cast<size_t>(M) * static_cast<size_t>(w->d.N) * 4)
+        return fail(MQ_ERR_INVALID_ARG, "workspace smaller than M*N*4 bytes");
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
+    if (dev != w->device)
+        return fail(MQ_ERR_INVALID_ARG, "the current device is not the device that packed the weight");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float *part = static_cast<float *>(workspace);
+    mq_status st = (M <= 16) ? launch_decode(w, X, static_cast<int>(M), Y, s, part)
+                             : launch_prefill(w, X, M, Y, s, part);
+    if (st) return st;
+    return launch_residual_merge(w, X, M, part, Y, s);
+}
+
+mq_status mq_linear(const mq_weight *w, const void *X, int64_t M, void *Y, mq_stream stream) {
+    return mq_linear_path(w, X, M, Y, stream, MQ_PATH_AUTO);
+}
+
+}  // extern "C"

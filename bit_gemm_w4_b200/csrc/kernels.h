@@ -1,0 +1,54 @@
+// Kernel launch interface between the C ABI (api.cpp) and the CUDA sources.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/mosaicq.h"
+
+struct mq_weight;
+
+namespace mq {
+
+// Device buffers of one packed weight (all on one GPU).
+struct DeviceWeight {
+    int64_t N, K, G, Gp, nnz;
+    const uint32_t *qweight;  // [N][K/8]
+    const uint32_t *sz;       // [N][Gp]
+    const int32_t *row_ptr;   // [N+1]
+    const uint16_t *col;      // [nnz] (+ padding)
+    const uint8_t *val;       // [(nnz+1)/2] (+ padding)
+    const uint16_t *rscale;   // [N]
+    int *err;                 // device error word
+};
+
+// Tensor maps and residual-slice sizes a kernel configuration needs; filled
+// by the host at pack time (see api.cpp).
+struct MapSet {
+    int bn = 0, gs = 0;
+    CUtensorMap w;   // qweight, box [bn rows][16 words]
+    CUtensorMap sz;  // sz, box [bn rows][gs words]
+    int64_t max_tile_nnz = 0;  // max residual entries over bn-row tiles
+};
+
+// Looks up (or builds) the MapSet for a tile shape of a handle.
+const MapSet *weight_maps(const mq_weight *w, int bn, int gs);
+const DeviceWeight &weight_device(const mq_weight *w);
+
+// Decode kernels (decode.cu): M in [1, 16]. With `partial` set the residual
+// is skipped and the dense base alone is written as fp32 to `partial`
+// (the unfused path's first half); else Y (bf16) gets the fused result.
+mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t stream,
+                        float *partial = nullptr);
+
+// Prefill kernel (prefill.cu): any M >= 1; `partial` as for decode.
+mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
+                         cudaStream_t stream, float *partial = nullptr);
+
+// Separate residual kernel (residual.cu): Y = bf16(partial + X * R^T).
+mq_status launch_residual_merge(const mq_weight *w, const void *X, int64_t M,
+                                const float *partial, void *Y, cudaStream_t stream);
+
+}  // namespace mq

@@ -1,0 +1,236 @@
+"""Thin ctypes binding of libmosaicq (include/mosaicq.h).
+
+Argument marshalling only: every step of the decomposition, packing and
+product runs inside the library (host C++ for packing, CUDA kernels for the
+product). PyTorch supplies device memory and streams. There is no fallback:
+if the library is missing or a call fails, an exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmosaicq.so")
+
+OK, INVALID_ARG, UNSUPPORTED, OUT_OF_MEMORY, CUDA, DEVICE_TIMEOUT = range(6)
+PATH_AUTO, PATH_DECODE, PATH_PREFILL = range(3)
+_PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "prefill": PATH_PREFILL}
+
+
+class MQError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: status {status} ({detail})")
+        self.status = status
+
+
+class _PackOpts(ctypes.Structure):
+    _fields_ = [("group_size", ctypes.c_int32), ("residual_density", ctypes.c_double)]
+
+
+class _Decomp(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("q", ctypes.c_void_p), ("s", ctypes.c_void_p), ("z", ctypes.c_void_p),
+                ("row_ptr", ctypes.c_void_p), ("col", ctypes.c_void_p),
+                ("qr", ctypes.c_void_p), ("sr", ctypes.c_void_p)]
+
+
+class _HostPacked(ctypes.Structure):
+    _fields_ = [("qweight", ctypes.c_void_p), ("sz", ctypes.c_void_p),
+                ("row_ptr", ctypes.c_void_p), ("col", ctypes.c_void_p),
+                ("val", ctypes.c_void_p), ("rscale", ctypes.c_void_p)]
+
+
+class _Info(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("K", ctypes.c_int64), ("nnz", ctypes.c_int64),
+                ("group_size", ctypes.c_int32), ("device", ctypes.c_int32),
+                ("device_bytes", ctypes.c_int64), ("max_row_nnz", ctypes.c_int64)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmosaicq.so is not built ({LIB_PATH}); run "
+                          "`python -m bit_gemm_w4_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    sig = {
+        "mq_pack": ([vp, i64, i64, ctypes.POINTER(_PackOpts), vp, ctypes.POINTER(vp)], st),
+        "mq_linear": ([vp, vp, i64, vp, vp], st),
+        "mq_linear_path": ([vp, vp, i64, vp, vp, ctypes.c_int], st),
+        "mq_linear_unfused": ([vp, vp, i64, vp, vp, ctypes.c_size_t, vp], st),
+        "mq_free": ([vp], None),
+        "mq_residual_nnz": ([i64, i64, ctypes.POINTER(_PackOpts), ctypes.POINTER(i64)], st),
+        "mq_pack_host": ([vp, i64, i64, ctypes.POINTER(_PackOpts), ctypes.POINTER(_HostPacked)], st),
+        "mq_pack_decomposed": ([ctypes.POINTER(_Decomp), vp, ctypes.POINTER(vp)], st),
+        "mq_get_info": ([vp, ctypes.POINTER(_Info)], st),
+        "mq_export": ([vp, ctypes.POINTER(_HostPacked)], st),
+        "mq_device_error": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], st),
+        "mq_strerror": ([st], ctypes.c_char_p),
+        "mq_last_error": ([], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        detail = _lib.mq_last_error().decode() or _lib.mq_strerror(status).decode()
+        raise MQError(status, where, detail)
+
+
+def _opts(rho: float, group: int = 128) -> _PackOpts:
+    return _PackOpts(group, float(rho))
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data if a.size else 0
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def residual_nnz(N: int, K: int, rho: float, group: int = 128) -> int:
+    out = ctypes.c_int64()
+    _check(_lib.mq_residual_nnz(N, K, ctypes.byref(_opts(rho, group)), ctypes.byref(out)),
+           "mq_residual_nnz")
+    return out.value
+
+
+def _alloc_packed(N: int, K: int, nnz: int):
+    arrs = dict(qweight=np.zeros((N, K // 8), np.uint32), sz=np.zeros((N, K // 128), np.uint32),
+                row_ptr=np.zeros(N + 1, np.int32), col=np.zeros(nnz, np.uint16),
+                val=np.zeros((nnz + 1) // 2, np.uint8), rscale=np.zeros(N, np.uint16))
+    hp = _HostPacked(*(_ptr(arrs[k]) for k in
+                       ("qweight", "sz", "row_ptr", "col", "val", "rscale")))
+    return arrs, hp
+
+
+def pack_host(W: np.ndarray, rho: float, group: int = 128) -> dict:
+    """Decompose and pack on the host (no CUDA call). Returns the packed arrays."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    nnz = residual_nnz(N, K, rho, group)
+    arrs, hp = _alloc_packed(N, K, nnz)
+    _check(_lib.mq_pack_host(_ptr(W), N, K, ctypes.byref(_opts(rho, group)), ctypes.byref(hp)),
+           "mq_pack_host")
+    return arrs
+
+
+class Weight:
+    """A packed weight on the current CUDA device (owns its device buffers)."""
+
+    def __init__(self, handle: int):
+        self._h = handle
+
+    @classmethod
+    def pack(cls, W: np.ndarray, rho: float, group: int = 128, stream=None) -> "Weight":
+        W = np.ascontiguousarray(W, dtype=np.float32)
+        N, K = W.shape
+        h = ctypes.c_void_p()
+        _check(_lib.mq_pack(_ptr(W), N, K, ctypes.byref(_opts(rho, group)), _stream(stream),
+                            ctypes.byref(h)), "mq_pack")
+        return cls(h.value)
+
+    @classmethod
+    def pack_decomposed(cls, d: dict, stream=None) -> "Weight":
+        """Pack a decomposition given as arrays (q u8 [N,K], s/z fp16 [N,G],
+        row_ptr, col, qr, sr fp16 [N])."""
+        N, K = int(d["N"]), int(d["K"])
+        keep = dict(
+            q=np.ascontiguousarray(d["q"], np.uint8),
+            s=np.ascontiguousarray(np.asarray(d["s"], np.float16).view(np.uint16)),
+            z=np.ascontiguousarray(np.asarray(d["z"], np.float16).view(np.uint16)),
+            row_ptr=np.ascontiguousarray(d["row_ptr"], np.int64),
+            col=np.ascontiguousarray(d["col"], np.int32),
+            qr=np.ascontiguousarray(d["qr"], np.int8),
+            sr=np.ascontiguousarray(np.asarray(d["sr"], np.float16).view(np.uint16)))
+        dc = _Decomp(N, K, *(_ptr(keep[k]) for k in ("q", "s", "z", "row_ptr", "col", "qr", "sr")))
+        h = ctypes.c_void_p()
+        _check(_lib.mq_pack_decomposed(ctypes.byref(dc), _stream(stream), ctypes.byref(h)),
+               "mq_pack_decomposed")
+        return cls(h.value)
+
+    @property
+    def handle(self) -> int:
+        return self._h
+
+    def info(self) -> dict:
+        i = _Info()
+        _check(_lib.mq_get_info(self._h, ctypes.byref(i)), "mq_get_info")
+        return {f: getattr(i, f) for f, _ in _Info._fields_}
+
+    def linear(self, X, Y=None, *, stream=None, path: str = "auto"):
+        """Y = X @ W_hat^T for bf16 X [M, K] on the packing device."""
+        import torch
+        info = self.info()
+        if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != info["K"]:
+            raise ValueError("X must be a bf16 [M, K] tensor")
+        X = X.contiguous()
+        if Y is None:
+            Y = torch.empty((X.shape[0], info["N"]), dtype=torch.bfloat16, device=X.device)
+        self.linear_raw(X.data_ptr(), X.shape[0], Y.data_ptr(), stream=stream, path=path)
+        return Y
+
+    def linear_raw(self, x_ptr: int, M: int, y_ptr: int, *, stream=None, path: str = "auto"):
+        _check(_lib.mq_linear_path(self._h, x_ptr, M, y_ptr, _stream(stream), _PATHS[path]),
+               "mq_linear")
+
+    def linear_unfused(self, X, Y=None, workspace=None, *, stream=None):
+        """The split comparison path: dense kernel into an fp32 workspace,
+        then a separate residual kernel (caller-owned workspace of M*N fp32)."""
+        import torch
+        info = self.info()
+        X = X.contiguous()
+        M = X.shape[0]
+        if Y is None:
+            Y = torch.empty((M, info["N"]), dtype=torch.bfloat16, device=X.device)
+        if workspace is None:
+            workspace = torch.empty((M, info["N"]), dtype=torch.float32, device=X.device)
+        _check(_lib.mq_linear_unfused(self._h, X.data_ptr(), M, Y.data_ptr(),
+                                      workspace.data_ptr(),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream(stream)), "mq_linear_unfused")
+        return Y
+
+    def export(self) -> dict:
+        info = self.info()
+        arrs, hp = _alloc_packed(info["N"], info["K"], info["nnz"])
+        _check(_lib.mq_export(self._h, ctypes.byref(hp)), "mq_export")
+        return arrs
+
+    def device_error(self, stream=None) -> int:
+        code = ctypes.c_int32()
+        st = _lib.mq_device_error(self._h, _stream(stream), ctypes.byref(code))
+        if st not in (OK, DEVICE_TIMEOUT):
+            _check(st, "mq_device_error")
+        return code.value
+
+    def free(self):
+        if self._h:
+            _lib.mq_free(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass

@@ -1,0 +1,185 @@
+/*
+ * mosaicq.h - C ABI of libmosaicq, a B200 (sm_100a) fused W4 + sparse-residual
+ * linear layer.
+ *
+ * Method: MosaicQuant (gist.science/paper/2606.15652, "Methodology").
+ *   1. Inlier-Outlier Disaggregation: a weight matrix W is split as
+ *      W ~= Q(W) + R, a dense 4-bit base Q that captures the inliers and a
+ *      sparse 4-bit residual R that compensates the quantization error the
+ *      outliers leave; both parts stay 4-bit.
+ *   3. ZipperEngine: the residual is computed inside the dense 4-bit GEMM
+ *      kernel instead of a separate kernel that would reload activations and
+ *      merge partial outputs; dense compute, sparse compensation and the
+ *      reduction-add run as one pipelined pass.
+ *   Problem statement as this library reads it: build the 4-bit form of W
+ *   once (mq_pack), then compute Y = X * W_hat^T many times (mq_linear).
+ *
+ * Encoding (the pages fix none; this library fixes it):
+ *   base     int4 asymmetric, group 128 along K, one fp16 scale s and one
+ *            fp16 zero point z (an integer 0..15) per (row, group):
+ *            deq = (q - z) * s.
+ *   residual per-row CSR of int4 codes q_r in [-8, 7] with one fp16 scale
+ *            s_r per row; row n keeps its k_n = floor(rho*K + 0.5) largest
+ *            |W - deq| entries (ties to the smaller column).
+ *            W_hat = deq + scatter(q_r * s_r).
+ *   product  exact products, fp32 accumulation, bf16 output (RNE).
+ *
+ * Conventions for every call:
+ *   - Status codes are returned; nothing aborts. mq_last_error() gives a
+ *     one-line reason for the most recent failure on the calling thread.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *   - Host pointers are CPU memory owned by the caller; device pointers are
+ *     CUDA global memory on the device that packed the weight.
+ *   - mq_linear* never allocate; mq_pack / mq_pack_decomposed own every
+ *     device buffer of a handle until mq_free.
+ *   - There is no CPU fallback: a missing or unusable GPU is an error.
+ */
+#ifndef MOSAICQ_H
+#define MOSAICQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *mq_stream; /* identical to cudaStream_t */
+typedef struct mq_weight mq_weight;    /* opaque; owns one packed W on one GPU */
+
+typedef enum {
+    MQ_OK = 0,
+    MQ_ERR_INVALID_ARG = 1,    /* bad pointer, size, value, alignment or device */
+    MQ_ERR_UNSUPPORTED = 2,    /* a valid request this build does not serve */
+    MQ_ERR_OUT_OF_MEMORY = 3,  /* a device or host allocation failed */
+    MQ_ERR_CUDA = 4,           /* a CUDA runtime / driver call failed */
+    MQ_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up a bounded wait */
+} mq_status;
+
+/* Which kernel mq_linear_path runs. MQ_PATH_AUTO is what mq_linear does:
+ * DECODE for M <= 16, PREFILL otherwise. */
+typedef enum {
+    MQ_PATH_AUTO = 0,
+    MQ_PATH_DECODE = 1,  /* register dequant + mma.sync, fused CSR walk; M <= 16 */
+    MQ_PATH_PREFILL = 2  /* tcgen05 / TMEM / TMA tensor-core kernel; any M >= 1 */
+} mq_path;
+
+typedef struct {
+    int32_t group_size;      /* must be 128, else MQ_ERR_UNSUPPORTED */
+    double residual_density; /* rho in [0, 1]; k_n = floor(rho*K + 0.5) per row */
+} mq_pack_opts;
+
+/* One decomposition in unpacked host form (caller-owned arrays). */
+typedef struct {
+    int64_t N, K;            /* rows (output features), columns (inputs) */
+    const uint8_t *q;        /* [N][K] base codes 0..15 */
+    const uint16_t *s;       /* [N][K/128] fp16 bits of the group scales (finite) */
+    const uint16_t *z;       /* [N][K/128] fp16 bits of the zero points (integers 0..15) */
+    const int64_t *row_ptr;  /* [N+1] residual CSR offsets: row_ptr[0] = 0, non-decreasing */
+    const int32_t *col;      /* [nnz] residual columns, strictly ascending per row, < K */
+    const int8_t *qr;        /* [nnz] residual codes in [-8, 7] */
+    const uint16_t *sr;      /* [N] fp16 bits of the residual scales (finite) */
+} mq_decomp;
+
+/* Caller-owned host buffers of the packed layout. Element counts: qweight
+ * N*K/8, sz N*K/128, row_ptr N+1, col nnz, val (nnz+1)/2, rscale N. */
+typedef struct {
+    uint32_t *qweight; /* word w of row n: bits [4j,4j+4) = q[n][8w + pi(j)],
+                          pi = (0,2,4,6,1,3,5,7) */
+    uint32_t *sz;      /* fp16 bits of s (low half) | fp16 bits of z (high half) */
+    int32_t *row_ptr;  /* CSR offsets */
+    uint16_t *col;     /* CSR columns */
+    uint8_t *val;      /* entry e: byte e>>1, low nibble when e is even;
+                          two's complement int4; an odd tail pads with 0 */
+    uint16_t *rscale;  /* fp16 bits of s_r */
+} mq_host_packed;
+
+typedef struct {
+    int64_t N, K, nnz;
+    int32_t group_size;
+    int32_t device;        /* CUDA ordinal that holds the buffers */
+    int64_t device_bytes;  /* device memory the handle owns */
+    int64_t max_row_nnz;   /* largest residual row */
+} mq_info;
+
+/* Decompose fp32 W[N][K] (host, row-major), pack it and upload it to the
+ * current device on `stream`. Returns after the upload completed; W may be
+ * freed then. *out = NULL on any error.
+ * Errors: INVALID_ARG for NULL pointers, N or K <= 0, K % 128 != 0,
+ * K > 65536, rho outside [0, 1], NaN/Inf in W, a scale that overflows fp16;
+ * UNSUPPORTED for group_size != 128; OUT_OF_MEMORY; CUDA. */
+mq_status mq_pack(const float *W_host, int64_t N, int64_t K,
+                  const mq_pack_opts *opts, mq_stream stream, mq_weight **out);
+
+/* Y[M][N] = X[M][K] * W_hat^T on `stream`, asynchronously: no host sync, no
+ * allocation. X and Y are bf16, row-major, device memory of the packing
+ * device, 16-byte aligned; Y is overwritten and must not overlap X. The
+ * handle is read-only here, so concurrent calls on different streams are
+ * safe. M = 0 launches nothing.
+ * Errors: INVALID_ARG for a NULL handle, NULL X/Y with M > 0, M < 0,
+ * misaligned X/Y or a current device other than the packing device; CUDA
+ * when a launch fails. */
+mq_status mq_linear(const mq_weight *w, const void *X_dev, int64_t M,
+                    void *Y_dev, mq_stream stream);
+
+/* As mq_linear with an explicit kernel choice. UNSUPPORTED for
+ * MQ_PATH_DECODE with M > 16. */
+mq_status mq_linear_path(const mq_weight *w, const void *X_dev, int64_t M,
+                         void *Y_dev, mq_stream stream, mq_path path);
+
+/* The split execution the fused pass avoids ("Methodology" 3.: a separate
+ * residual kernel reloads the activations and merges partial outputs), kept
+ * as the comparison the fused kernels are measured against. The dense base
+ * kernel writes fp32 partial outputs into `workspace`, then a second kernel
+ * re-reads X, adds the residual to the partials and writes bf16 Y (one
+ * rounding, so the result meets the same bounds as mq_linear).
+ * workspace: caller-owned device memory of at least M*N*4 bytes, 16-byte
+ * aligned, not shared with a concurrent call. Errors as mq_linear, plus
+ * INVALID_ARG for a NULL, misaligned or too small workspace. */
+mq_status mq_linear_unfused(const mq_weight *w, const void *X_dev, int64_t M,
+                            void *Y_dev, void *workspace, size_t workspace_bytes,
+                            mq_stream stream);
+
+/* Release every buffer of the handle. NULL-safe. Waits for no stream: the
+ * caller makes sure no call using the handle is still in flight. */
+void mq_free(mq_weight *w);
+
+/* --- support for tests and benchmarks (not needed for inference) --- */
+
+/* Residual entries a pack with these options produces: N * k_n. */
+mq_status mq_residual_nnz(int64_t N, int64_t K, const mq_pack_opts *opts,
+                          int64_t *nnz);
+
+/* Decompose and pack on the host only (no CUDA call at all) into caller
+ * buffers sized with mq_residual_nnz. Same validation as mq_pack. */
+mq_status mq_pack_host(const float *W_host, int64_t N, int64_t K,
+                       const mq_pack_opts *opts, mq_host_packed *out);
+
+/* Pack a given decomposition (validated: code ranges, integer zero points
+ * 0..15, finite scales, CSR structure) and upload it like mq_pack. */
+mq_status mq_pack_decomposed(const mq_decomp *d, mq_stream stream,
+                             mq_weight **out);
+
+/* Shape and footprint of a handle. */
+mq_status mq_get_info(const mq_weight *w, mq_info *out);
+
+/* Copy the packed bytes of a handle back into caller host buffers (sized
+ * from mq_get_info). Synchronous: waits for the device. */
+mq_status mq_export(const mq_weight *w, mq_host_packed *out);
+
+/* Read and clear the handle's device error word: 0 when every kernel since
+ * the last read finished its waits, else the code of the wait that gave up.
+ * Synchronizes `stream`. Returns MQ_ERR_DEVICE_TIMEOUT when non-zero. */
+mq_status mq_device_error(const mq_weight *w, mq_stream stream, int32_t *code);
+
+/* Static text for a status code. */
+const char *mq_strerror(mq_status s);
+
+/* One-line reason for the calling thread's most recent failure ("" if none). */
+const char *mq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOSAICQ_H */

@@ -31,3 +31,20 @@ def read_golden(name):
 @pytest.fixture
 def golden():
     return read_golden
+
+
+@pytest.fixture(scope="session")
+def mq():
+    """The ctypes binding, building libmosaicq.so first if it is stale."""
+    from bit_gemm_w4_b200 import build
+    build.build()
+    from bit_gemm_w4_b200 import mosaicq
+    return mosaicq
+
+
+@pytest.fixture(scope="session")
+def cuda(mq):
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")

@@ -1,0 +1,179 @@
+"""GPU parity: the CUDA path against the fp64 oracle on the same seeded
+inputs, through the C ABI. Bounds (oracle/tolerance.py): normalized error
+<= 2e-3 and relative error <= 1e-2 where |y| > 1e-3; packed bytes bit-exact.
+
+MosaicQuant "Methodology" 1. (W ~= Q(W) + R, both 4-bit) and 3. (the fused
+dense + sparse pass ending in one reduction-add)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_gemm_w4_b200 import synth
+from gpu_util import oracle_check
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(mq, W, X, rho, path="auto"):
+    w = mq.Weight.pack(W, rho)
+    Y = w.linear(X.cuda(), path=path)
+    torch.cuda.synchronize()
+    assert w.device_error() == 0
+    return w, Y
+
+
+def _bytes_equal(got, want):
+    for k in ("qweight", "sz", "row_ptr", "col", "val", "rscale"):
+        a, b = np.asarray(got[k]), np.ascontiguousarray(want[k])
+        assert a.shape == b.shape and np.array_equal(a.view(np.uint8), b.view(np.uint8)), k
+
+
+def test_tiny_workload(mq, cuda):
+    W, X, rho = synth.workload_inputs("tiny")
+    w, Y = _run(mq, W, X, rho)
+    d = oracle.decompose(W, rho)
+    _bytes_equal(w.export(), oracle.pack(d))
+    r = oracle_check(Y, X, d)
+    assert r["ok"], r
+
+
+@pytest.mark.parametrize("shape", [0, 1, 2])
+def test_7b_decode_workload(mq, cuda, shape):
+    W, X, rho = synth.workload_inputs("7b_decode", shape)
+    w, Y = _run(mq, W, X, rho)
+    d = oracle.decompose(W, rho)
+    _bytes_equal(w.export(), oracle.pack(d))
+    r = oracle_check(Y, X, d)
+    assert r["ok"], r
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 9, 12, 16])
+def test_decode_token_counts_ragged_rows(mq, cuda, M):
+    W = synth.weight(200, 1024, std=0.02, outlier_frac=0.01, seed=M)
+    X = synth.activations(M, 1024, seed=100 + M, channels=4, mult=20.0)
+    w, Y = _run(mq, W, X, 0.02, path="decode")
+    r = oracle_check(Y, X, oracle.decompose(W, 0.02))
+    assert r["ok"], r
+
+
+@pytest.mark.parametrize("M", [17, 40, 129])
+def test_prefill_token_counts(mq, cuda, M):
+    W = synth.weight(136, 512, std=0.02, outlier_frac=0.01, seed=M)
+    X = synth.activations(M, 512, seed=200 + M, channels=8, mult=30.0)
+    w, Y = _run(mq, W, X, 0.01, path="auto")
+    r = oracle_check(Y, X, oracle.decompose(W, 0.01))
+    assert r["ok"], r
+
+
+@pytest.mark.parametrize("path", ["decode", "prefill", "unfused"])
+@pytest.mark.parametrize("M", [1, 16])
+def test_every_path_small(mq, cuda, path, M):
+    W = synth.weight(264, 896, std=0.02, outlier_frac=0.01, seed=3)
+    X = synth.activations(M, 896, seed=4, channels=4, mult=20.0)
+    if path == "unfused":
+        w = mq.Weight.pack(W, 0.01)
+        Y = w.linear_unfused(X.cuda())
+        torch.cuda.synchronize()
+    else:
+        w, Y = _run(mq, W, X, 0.01, path=path)
+    r = oracle_check(Y, X, oracle.decompose(W, 0.01))
+    assert r["ok"], (path, r)
+
+
+@pytest.mark.parametrize("M", [1, 8, 40])
+def test_unfused_matches_fused(mq, cuda, M):
+    W = synth.weight(300, 1024, std=0.02, outlier_frac=0.01, seed=M)
+    X = synth.activations(M, 1024, seed=9, channels=4, mult=20.0).cuda()
+    w = mq.Weight.pack(W, 0.03)
+    Yf = w.linear(X)
+    Yu = w.linear_unfused(X)
+    torch.cuda.synchronize()
+    r = oracle_check(Yu, X.cpu(), oracle.decompose(W, 0.03))
+    assert r["ok"], r
+    # both round an fp32 result once; they may differ by one bf16 ulp
+    diff = (Yf.float() - Yu.float()).abs()
+    assert float((diff / Yf.float().abs().clamp_min(1e-3)).max()) < 2 ** -7
+
+
+@pytest.mark.parametrize("rho", [0.0, 0.04])
+def test_density_zero_and_dense_residual(mq, cuda, rho):
+    W = synth.weight(128, 4096, std=0.02, outlier_frac=0.005, seed=5)
+    X = synth.activations(8, 4096, seed=6, channels=4, mult=20.0)
+    w, Y = _run(mq, W, X, rho)
+    r = oracle_check(Y, X, oracle.decompose(W, rho))
+    assert r["ok"], r
+
+
+def test_single_group_and_tiny_n(mq, cuda):
+    W = synth.weight(8, 128, std=0.02, outlier_frac=0.02, seed=7)
+    X = synth.activations(3, 128, seed=8)
+    w, Y = _run(mq, W, X, 0.05)
+    r = oracle_check(Y, X, oracle.decompose(W, 0.05))
+    assert r["ok"], r
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_sweep_decomposition_dense_clustered(mq, cuda, M):
+    dd = synth.sweep_decomposition(256, 4096, 164, seed=11)
+    w = mq.Weight.pack_decomposed(dd)
+    X = synth.activations(M, 4096, seed=12)
+    Y = w.linear(X.cuda())
+    torch.cuda.synchronize()
+    d = oracle.from_arrays(dd)
+    _bytes_equal(w.export(), oracle.pack(d))
+    r = oracle_check(Y, X, d)
+    assert r["ok"], r
+
+
+def test_argument_errors(mq, cuda):
+    W = synth.weight(16, 128, std=0.02, outlier_frac=0.0, seed=1)
+    w = mq.Weight.pack(W, 0.01)
+    X = torch.zeros((2, 128), dtype=torch.bfloat16, device=cuda)
+    Y = torch.zeros((2, 16), dtype=torch.bfloat16, device=cuda)
+    w.linear_raw(X.data_ptr(), 0, Y.data_ptr())                      # M = 0: no-op
+    with pytest.raises(mq.MQError) as e:
+        w.linear_raw(X.data_ptr() + 2, 2, Y.data_ptr())              # misaligned X
+    assert e.value.status == mq.INVALID_ARG
+    with pytest.raises(mq.MQError) as e:
+        w.linear_raw(X.data_ptr(), -1, Y.data_ptr())
+    assert e.value.status == mq.INVALID_ARG
+    with pytest.raises(mq.MQError) as e:
+        w.linear_raw(X.data_ptr(), 17, Y.data_ptr(), path="decode")  # decode serves M <= 16
+    assert e.value.status == mq.UNSUPPORTED
+    with pytest.raises(mq.MQError):
+        w.linear_raw(0, 2, Y.data_ptr())
+    small = torch.zeros(4, dtype=torch.float32, device=cuda)
+    with pytest.raises(mq.MQError) as e:
+        w.linear_unfused(X, Y, small)                                # workspace too small
+    assert e.value.status == mq.INVALID_ARG
+
+
+def test_70b_mlp_full_size_sampled_rows(mq, cuda):
+    cfg = synth.WORKLOADS["70b_mlp"]
+    N, K = cfg["shapes"][0]
+    W, X, rho = synth.workload_inputs("70b_mlp")
+    w, Y = _run(mq, W, X, rho)
+    rows = np.unique(np.concatenate([np.arange(0, 40), np.arange(N - 24, N),
+                                     np.random.default_rng(0).choice(N, 64, replace=False)]))
+    d = oracle.decompose(np.ascontiguousarray(W[rows]), rho)
+    ex = w.export()
+    want = oracle.pack(d)
+    assert np.array_equal(ex["qweight"][rows], want["qweight"])
+    assert np.array_equal(ex["sz"][rows], want["sz"])
+    assert np.array_equal(ex["rscale"][rows], want["rscale"])
+    r = oracle_check(Y[:, rows], X, d)
+    assert r["ok"], r
+
+
+def test_prefill_full_size_sampled_rows(mq, cuda):
+    cfg = synth.WORKLOADS["prefill"]
+    N, K = cfg["shapes"][0]
+    W, X, rho = synth.workload_inputs("prefill")
+    w, Y = _run(mq, W, X, rho)
+    rows = np.unique(np.concatenate([np.arange(0, 32), np.arange(N - 16, N),
+                                     np.random.default_rng(1).choice(N, 48, replace=False)]))
+    d = oracle.decompose(np.ascontiguousarray(W[rows]), rho)
+    r = oracle_check(Y[:, rows], X, d)
+    assert r["ok"], r

@@ -1,0 +1,63 @@
+"""The library's host decomposition + packing equals the oracle's, byte for
+byte (MosaicQuant "Methodology" 1.: W ~= Q(W) + R, both parts 4-bit, in the
+encoding this library fixes). Runs without a GPU (mq_pack_host)."""
+
+import numpy as np
+import pytest
+
+import oracle
+from bit_gemm_w4_b200 import synth
+
+
+def _same(mq, W, rho):
+    got = mq.pack_host(W, rho)
+    want = oracle.pack(oracle.decompose(W, rho))
+    for k in ("qweight", "sz", "row_ptr", "col", "val", "rscale"):
+        a, b = np.asarray(got[k]), np.asarray(want[k])
+        assert a.shape == b.shape, k
+        assert a.dtype.itemsize == b.dtype.itemsize, k
+        assert np.array_equal(a.view(np.uint8), np.ascontiguousarray(b).view(np.uint8)), k
+
+
+def test_tiny_workload(mq):
+    W, _, rho = synth.workload_inputs("tiny")
+    _same(mq, W, rho)
+
+
+def test_7b_qkvo_workload(mq):
+    W, _, rho = synth.workload_inputs("7b_decode", 0)
+    _same(mq, W, rho)
+
+
+def test_down_shape_rows(mq):
+    W, _, rho = synth.workload_inputs("7b_decode", 2, rows=np.arange(0, 4096, 97))
+    _same(mq, W, rho)
+
+
+def test_70b_like_rows(mq):
+    rng = np.random.default_rng(0)
+    W = (rng.standard_normal((5, 8192)) * 0.015).astype(np.float32)
+    W[:, rng.choice(8192, 32, replace=False)] = (0.2 * rng.standard_t(3, (5, 32))).astype(np.float32)
+    _same(mq, W, 0.01)
+
+
+@pytest.mark.parametrize("rho", [0.0, 0.25, 1.0])
+def test_density_extremes(mq, rho):
+    W = synth.weight(24, 256, std=0.02, outlier_frac=0.02, seed=9)
+    _same(mq, W, rho)
+
+
+def test_ties_zeros_and_constants(mq):
+    W = np.zeros((6, 256), np.float32)
+    W[1] = 0.5                                        # constant row
+    W[2, ::3] = 0.25                                  # many equal errors
+    W[3] = np.tile(np.float32([0.1, -0.1, 0.3, 0.0]), 64)
+    W[4, 0] = 1e-9                                    # scale floor 2^-24
+    W[5] = np.abs(np.random.default_rng(1).standard_normal(256)).astype(np.float32)
+    _same(mq, W, 0.05)
+
+
+def test_subnormal_scales(mq):
+    rng = np.random.default_rng(2)
+    W = (rng.standard_normal((8, 128)) * 1e-5).astype(np.float32)
+    _same(mq, W, 0.03)
