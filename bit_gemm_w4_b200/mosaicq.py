@@ -61,6 +61,7 @@ def _load():
         "mq_linear": ([vp, vp, i64, vp, vp], st),
         "mq_linear_path": ([vp, vp, i64, vp, vp, ctypes.c_int], st),
         "mq_linear_unfused": ([vp, vp, i64, vp, vp, ctypes.c_size_t, vp], st),
+        "mq_linear_unfused_noalloc": ([vp, vp, i64, vp, vp], st),
         "mq_free": ([vp], None),
         "mq_residual_nnz": ([i64, i64, ctypes.POINTER(_PackOpts), ctypes.POINTER(i64)], st),
         "mq_pack_host": ([vp, i64, i64, ctypes.POINTER(_PackOpts), ctypes.POINTER(_HostPacked)], st),
@@ -209,6 +210,18 @@ class Weight:
                                       workspace.data_ptr(),
                                       workspace.numel() * workspace.element_size(),
                                       _stream(stream)), "mq_linear_unfused")
+        return Y
+
+    def linear_unfused_noalloc(self, X, Y=None, *, stream=None):
+        """The split comparison path with the library's built-in scratch (no
+        workspace argument and no device allocation by the library)."""
+        import torch
+        info = self.info()
+        X = X.contiguous()
+        if Y is None:
+            Y = torch.empty((X.shape[0], info["N"]), dtype=torch.bfloat16, device=X.device)
+        _check(_lib.mq_linear_unfused_noalloc(self._h, X.data_ptr(), X.shape[0], Y.data_ptr(),
+                                              _stream(stream)), "mq_linear_unfused_noalloc")
         return Y
 
     def export(self) -> dict:

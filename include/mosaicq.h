@@ -140,6 +140,28 @@ mq_status mq_linear_unfused(const mq_weight *w, const void *X_dev, int64_t M,
                             void *Y_dev, void *workspace, size_t workspace_bytes,
                             mq_stream stream);
 
+/* Largest M*N mq_linear_unfused_noalloc accepts (its built-in scratch). */
+#define MQ_UNFUSED_NOALLOC_MAX_OUTPUTS (2 * 1024 * 1024)
+
+/* mq_linear_unfused for callers that cannot allocate device memory. The
+ * paper has no counterpart: this is a deployment variant of the unfused
+ * comparison path. Some callers cannot hand out a workspace or call
+ * cudaMalloc: code that runs inside a fixed memory budget or a pool it does
+ * not own, plugins that only receive their input and output buffers, hosts
+ * that route every device allocation through their own allocator. This call
+ * keeps the M*N fp32 partial outputs in a fixed array inside the library
+ * (MQ_UNFUSED_NOALLOC_MAX_OUTPUTS floats, 8 MiB, held on every GPU that
+ * loads the library until the process exits) and performs no allocation of
+ * any kind. Results match mq_linear_unfused.
+ * The first call on each device looks up the array's device address with
+ * that device current; make it before any stream capture. All calls on a
+ * device share the array, which keeps the last call's contents (nothing in
+ * it needs to start at zero); calls whose GPU work overlaps in time race.
+ * Errors as mq_linear, plus INVALID_ARG when M*N exceeds
+ * MQ_UNFUSED_NOALLOC_MAX_OUTPUTS and CUDA when the address lookup fails. */
+mq_status mq_linear_unfused_noalloc(const mq_weight *w, const void *X_dev,
+                                    int64_t M, void *Y_dev, mq_stream stream);
+
 /* Release every buffer of the handle. NULL-safe. Waits for no stream: the
  * caller makes sure no call using the handle is still in flight. */
 void mq_free(mq_weight *w);
