@@ -183,7 +183,8 @@ def time_graph_steps(torch, ds: DecodeSet, steps: int, warmup: int, stream, chun
     g_rem = capture(rem) if rem else None
     # settle clocks under the same load before the timed region
     t_end = time.time() + 0.5
-    with ClockSampler(sampler_gpu) as clk:
+    # CUDAGraph.replay() launches on the current stream: make it `stream`
+    with ClockSampler(sampler_gpu) as clk, torch.cuda.stream(stream):
         while time.time() < t_end:
             (g or g_rem).replay()
         torch.cuda.synchronize()
@@ -212,15 +213,16 @@ def time_per_shape(torch, ds: DecodeSet, stream, n: int = 48):
         with torch.cuda.graph(g, stream=stream):
             for k in range(n):
                 ds.launch(k % copies, i, stream)
-        g.replay()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(5):
+        with torch.cuda.stream(stream):
             g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(5):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
         out.append(e0.elapsed_time(e1) / (5 * n))
     return out
 

@@ -27,8 +27,10 @@ struct mq_weight {
     std::vector<int32_t> host_row_ptr;  // for residual tile statistics
     mutable std::mutex maps_mu;
     mutable std::vector<mq::MapSet *> maps;
+    mutable mq::PrefillMaps *pmaps = nullptr;
     ~mq_weight() {
         for (auto *m : maps) delete m;
+        delete pmaps;
     }
 };
 
@@ -62,6 +64,21 @@ bool encode_2d_u32(CUtensorMap *map, const void *base, uint64_t inner, uint64_t 
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, const void *base,
+               uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * static_cast<uint64_t>(esize)};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -176,6 +193,30 @@ const MapSet *weight_maps(const mq_weight *w, int bn, int gs) {
     }
     w->maps.push_back(m);
     return m;
+}
+
+const PrefillMaps *prefill_maps(const mq_weight *w) {
+    std::lock_guard<std::mutex> lock(w->maps_mu);
+    if (w->pmaps) return w->pmaps;
+    PrefillMaps *m = new (std::nothrow) PrefillMaps();
+    if (!m) return nullptr;
+    const DeviceWeight &d = w->d;
+    if (d.Gp > 256 ||
+        !encode_2d(&m->w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, d.qweight, d.K / 8, d.N, 8, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_2d(&m->sz, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, d.sz, d.Gp, d.N,
+                   static_cast<uint32_t>(d.Gp), 128, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        delete m;
+        fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill maps");
+        return nullptr;
+    }
+    w->pmaps = m;
+    return m;
+}
+
+bool encode_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K) {
+    return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, static_cast<uint64_t>(K),
+                     static_cast<uint64_t>(M), 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace mq

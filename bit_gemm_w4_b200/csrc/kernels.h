@@ -35,6 +35,16 @@ struct MapSet {
 
 // Looks up (or builds) the MapSet for a tile shape of a handle.
 const MapSet *weight_maps(const mq_weight *w, int bn, int gs);
+
+// Tensor maps of the prefill kernel (built once per handle).
+struct PrefillMaps {
+    CUtensorMap w;   // qweight, box [128 rows][8 words] (64 columns)
+    CUtensorMap sz;  // sz, box [128 rows][Gp words]
+};
+const PrefillMaps *prefill_maps(const mq_weight *w);
+
+// bf16 X [M][K] row-major, box [128 rows][64 columns], 128-byte swizzle.
+bool encode_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K);
 const DeviceWeight &weight_device(const mq_weight *w);
 
 // Decode kernels (decode.cu): M in [1, 16]. With `partial` set the residual

@@ -177,3 +177,28 @@ def test_prefill_full_size_sampled_rows(mq, cuda):
     d = oracle.decompose(np.ascontiguousarray(W[rows]), rho)
     r = oracle_check(Y[:, rows], X, d)
     assert r["ok"], r
+
+
+@pytest.mark.parametrize("N,K,M,rho", [
+    (200, 128, 130, 0.02),      # one group, ragged rows and tokens
+    (136, 11008, 40, 0.005),    # 86 groups (padded scale rows), ragged rows
+    (300, 4096, 256, 0.01),     # two token tiles, three row tiles
+    (128, 512, 17, 0.0),        # no residual
+])
+def test_prefill_kernel_shapes(mq, cuda, N, K, M, rho):
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.01, seed=N + K)
+    X = synth.activations(M, K, seed=M, channels=8, mult=30.0)
+    w, Y = _run(mq, W, X, rho, path="prefill")
+    r = oracle_check(Y, X, oracle.decompose(W, rho))
+    assert r["ok"], r
+
+
+def test_prefill_kernel_dense_residual(mq, cuda):
+    dd = synth.sweep_decomposition(256, 4096, 164, seed=21)
+    w = mq.Weight.pack_decomposed(dd)
+    X = synth.activations(200, 4096, seed=22)
+    Y = w.linear(X.cuda(), path="prefill")
+    torch.cuda.synchronize()
+    assert w.device_error() == 0
+    r = oracle_check(Y, X, oracle.from_arrays(dd))
+    assert r["ok"], r
