@@ -204,8 +204,8 @@ const PrefillMaps *prefill_maps(const mq_weight *w) {
     if (d.Gp > 256 ||
         !encode_2d(&m->w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, d.qweight, d.K / 8, d.N, 8, 128,
                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_2d(&m->sz, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, d.sz, d.Gp, d.N,
-                   static_cast<uint32_t>(d.Gp), 128, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        !encode_2d(&m->sz, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, d.sz, d.Gp, d.N, 4, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE)) {
         delete m;
         fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill maps");
         return nullptr;

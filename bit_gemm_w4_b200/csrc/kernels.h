@@ -39,7 +39,7 @@ const MapSet *weight_maps(const mq_weight *w, int bn, int gs);
 // Tensor maps of the prefill kernel (built once per handle).
 struct PrefillMaps {
     CUtensorMap w;   // qweight, box [128 rows][8 words] (64 columns)
-    CUtensorMap sz;  // sz, box [128 rows][Gp words]
+    CUtensorMap sz;  // sz, box [128 rows][4 words]
 };
 const PrefillMaps *prefill_maps(const mq_weight *w);
 
