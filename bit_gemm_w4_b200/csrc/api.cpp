@@ -10,6 +10,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <new>
 #include <string>
@@ -201,11 +202,10 @@ const PrefillMaps *prefill_maps(const mq_weight *w) {
     PrefillMaps *m = new (std::nothrow) PrefillMaps();
     if (!m) return nullptr;
     const DeviceWeight &d = w->d;
+    m->pw = static_cast<int>(std::min<int64_t>(32, d.K / 8));
     if (d.Gp > 256 ||
-        !encode_2d(&m->w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, d.qweight, d.K / 8, d.N, 8, 128,
-                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_2d(&m->sz, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, d.sz, d.Gp, d.N, 4, 128,
-                   CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        !encode_2d(&m->w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, d.qweight, d.K / 8, d.N, m->pw, 128,
+                   m->pw == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE)) {
         delete m;
         fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill maps");
         return nullptr;
@@ -214,9 +214,19 @@ const PrefillMaps *prefill_maps(const mq_weight *w) {
     return m;
 }
 
-bool encode_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K) {
-    return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, static_cast<uint64_t>(K),
-                     static_cast<uint64_t>(M), 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+bool encode_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K, int chunks) {
+    // X [M][K] viewed as [K/64][M][64]: one box is `chunks` consecutive
+    // 64-column tiles [128 rows][64], each 128-byte swizzled
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(K / 64)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, 128};
+    cuuint32_t box[3] = {64, 128, static_cast<cuuint32_t>(chunks)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(X), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 }  // namespace mq

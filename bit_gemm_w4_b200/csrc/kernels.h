@@ -38,13 +38,14 @@ const MapSet *weight_maps(const mq_weight *w, int bn, int gs);
 
 // Tensor maps of the prefill kernel (built once per handle).
 struct PrefillMaps {
-    CUtensorMap w;   // qweight, box [128 rows][8 words] (64 columns)
-    CUtensorMap sz;  // sz, box [128 rows][4 words]
+    CUtensorMap w;  // qweight, box [128 rows][pw words]; 128-byte swizzle when pw = 32
+    int pw;         // words per row of a box: min(32, K / 8), four or two 64-column stages
 };
 const PrefillMaps *prefill_maps(const mq_weight *w);
 
-// bf16 X [M][K] row-major, box [128 rows][64 columns], 128-byte swizzle.
-bool encode_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K);
+// bf16 X [M][K] row-major as a 3D view [K/64][M][64]; one box holds `chunks`
+// consecutive [128 rows][64 columns] tiles, each 128-byte swizzled.
+bool encode_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K, int chunks);
 const DeviceWeight &weight_device(const mq_weight *w);
 
 // Decode kernels (decode.cu): M in [1, 16]. With `partial` set the residual

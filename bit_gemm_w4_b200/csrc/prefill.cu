@@ -6,32 +6,46 @@
 // compensation and the reduction-add run as one overlapped pipeline on
 // tensor cores, CUDA cores and HBM.
 //
-// One CTA computes a 128-token x 128-row output tile over all of K, in
-// stages of 64 columns, with warp roles:
-//   warp 0      TMA producer: the X tile [128 tokens][64] (128-byte swizzle)
-//               and the packed codes [128 rows][8 words] of each stage into
-//               a deep ring (S1 stages), plus the tile's scale/zero words
-//               once, as [groups/4][128 rows][4 words] boxes.
+// The kernel is persistent: one CTA per SM walks a contiguous range of
+// 128-row x 128-token output tiles (consecutive tiles share their weight
+// rows), each over all of K in stages of 64 columns; the pipelines below run
+// on across tile boundaries, so a tile's first stages load and dequantize
+// while the previous tile's last MMAs and epilogue finish. The weight is the MMA's A operand and lives in
+// tensor memory, X is the B operand and streams through shared memory
+// (D[row][token] = sum_k A[row][k] * X[token][k]), so the dequantized codes
+// never touch shared memory: the only shared-memory traffic per stage is the
+// TMA write of X and of the packed codes and the tensor core's read of X.
+// Warp roles:
+//   warp 0      TMA producer (one thread). One thread's copies complete one
+//               after another, so few large copies are issued: the X tiles
+//               [128 tokens][64] (128-byte swizzle) of CX consecutive stages
+//               per copy (X seen as a 3D tensor [K/64][M][64]) into a ring of
+//               XS slots, and the packed codes of four stages per copy
+//               ([128 rows][32 words], 128-byte swizzle) into two slots.
 //   warp 1      allocates tensor memory and issues tcgen05.mma (one thread).
 //   warps 2..9  epilogue, two per tensor-memory lane quadrant (thread =
-//               token), each owning 64 of the tile's 128 columns.
-//   warps 10..13 dequant, thread = weight row: the 8 packed words of the row
-//               become its 64 exact bf16 codes (q - z), written straight into
-//               the 128-byte-swizzled K-major operand layout; the row's
-//               residual entries of the stage are written as exact bf16
-//               codes q_r into a second operand tile (zeros elsewhere).
-// Per stage the MMA thread issues 4 K=16 steps of the dense tile into the
-// TMEM buffer of the current 128-column group and 4 steps of the residual
-// tile into a TMEM accumulator that spans all of K. Every product is exact
+//               weight row), each owning 64 of the tile's 128 tokens.
+//   warps 10..13 dequant, thread = weight row (its tensor-memory lane; scale
+//               and zero words and the CSR entries come through L1): the 8
+//               packed words of the row become its 64 exact bf16 codes
+//               (q - z), stored into a tensor-memory operand slot with one
+//               tcgen05.st. The row's residual entries of the stage are
+//               scattered as exact bf16 codes q_r into a shared-memory tile
+//               (128-byte swizzle, K-major) that is otherwise zero; when the
+//               slot comes round again only those entries are cleared.
+// Tensor memory (512 columns): the group partials D[2] at 0 / 128, the
+// residual accumulator R at 256, four 32-column operand slots at 384.
+// Per stage the MMA thread issues 4 K=16 steps of the dense codes (A from
+// tensor memory) into the TMEM buffer of the current 128-column group and,
+// when any of the tile's rows has a residual entry in the stage, 4 steps of
+// the residual tile (A from shared memory) into R. Every product is exact
 // (integer codes times bf16 x) and accumulates in fp32. When a group's two
-// stages are done the epilogue reads its partial sums from TMEM and adds
+// stages are done the epilogue reads its partial sums and adds
 // s[n][g] * partial to per-thread fp32 accumulators (the per-group rescale
-// the fp16 group scales require); the next group's MMAs run meanwhile into
-// the other buffer. After the last stage the residual accumulator is scaled
-// by s_r[n] and added (the reduction-add), and the tile is stored as bf16.
-// The residual's exact codes make it a second dense MMA per stage; rows
-// whose residual is empty still pay for it (the cost a block-sparse
-// residual allocation would avoid).
+// the fp16 group scales require; one scale per thread); the next group's
+// MMAs run meanwhile into the other buffer. After a tile's last stage R is
+// scaled by s_r[n] and added (the reduction-add) and the tile is stored as
+// bf16, while the next tile's MMAs already run.
 
 #include "common.cuh"
 #include "internal.h"
@@ -40,59 +54,58 @@
 namespace mq {
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 64;
-constexpr int MAX_S1 = 8;  // TMA ring depth (runtime S1 <= MAX_S1)
+constexpr int BM = 128;  // tokens per tile (the MMA's N)
+constexpr int BN = 128;  // weight rows per tile (the MMA's M, tensor-memory lanes)
+constexpr int BK = 64;
+constexpr int MAX_XS = 4;  // X ring slots (runtime XS <= MAX_XS)
 constexpr int THREADS = 448;
 constexpr int W_TMA = 0, W_MMA = 1, W_EPI0 = 2, W_DQ0 = 10;
-constexpr int EPI_WARPS = 8, EPI_COLS = BN / 2;  // two warps per lane quadrant
-constexpr int A_BYTES = BM * BK * 2;  // X tile
-constexpr int B_BYTES = BN * BK * 2;  // one dequantized operand tile
-constexpr int P_BYTES = BN * BK / 2;  // packed codes
-constexpr int T_BYTES = A_BYTES + P_BYTES;  // one TMA stage: A at 0, P after it
-constexpr int OFF_P = A_BYTES;
-constexpr int BB_BYTES = 2 * B_BYTES;  // one operand buffer: dense at 0, residual after
-constexpr uint32_t TMEM_COLS = 512;  // D[2] at 0 / 128, residual at 256
-static_assert(T_BYTES % 1024 == 0 && BB_BYTES % 1024 == 0, "1024-byte swizzle alignment");
+constexpr int EPI_WARPS = 8, EPI_TOK = BM / 2;  // two warps per lane quadrant
+constexpr int X_BYTES = BM * BK * 2;  // X tile
+constexpr int T_BYTES = X_BYTES;      // one TMA stage
+constexpr int PSLOT_BYTES = BN * 32 * 4;  // packed codes of up to four stages
+constexpr int NPSLOT = 2;
+constexpr int R_BYTES = BN * BK * 2;  // one residual code tile
+constexpr int NSLOT = 4;              // operand slots (dense in TMEM, residual in smem)
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t T_D = 0, T_R = 256, T_A = 384;  // column bases
+constexpr uint32_t A_SLOT = 32;                    // columns per operand slot
+static_assert(T_BYTES % 1024 == 0 && R_BYTES % 1024 == 0, "1024-byte swizzle alignment");
+static_assert(2 * T_BYTES >= BM * BN * 2, "the output tile is staged in the TMA ring");
 
 struct PrefillParams {
-    CUtensorMap tm_x;   // X [M][K] bf16, box [128][64], 128B swizzle
-    CUtensorMap tm_w;   // qweight [N][K/8] u32, box [128][8]
-    CUtensorMap tm_sz;  // sz [N][Gp] u32, box [128][4]
+    CUtensorMap tm_x;  // X [M][K] bf16, box [128][64], 128B swizzle
+    CUtensorMap tm_w;  // qweight [N][K/8] u32, box [128][8]
     const int32_t *row_ptr;
     const uint16_t *col;
     const uint8_t *val;
     const uint16_t *rscale;
+    const uint32_t *sz;  // [N][Gp] scale | zero << 16
     __nv_bfloat16 *Y;
     float *Yf;
     int *err;
     int M, N, K, G, Gp;
     int with_residual;
-    int csr_cap;  // residual entries the shared-memory slice holds (0: read global)
-    int S1;       // TMA ring depth
-    int S2;       // operand ring depth (2 or 3)
+    int XS;       // X ring slots
+    int CX;       // stages per X copy (2 or 4)
+    int pw;       // words per row of a packed-code box (32, or 16 when K = 128)
+    int m_tiles;  // token tiles; tile t covers rows (t / m_tiles) and tokens (t % m_tiles)
+    int tiles;
 };
 
 struct SmemLayout {
-    int bring, sz, sfr, srs, rflag, bars, tmem_slot, abort, col, val, total;
-    __host__ __device__ SmemLayout(int S1, int S2, int Gp, int csr_cap) {
-        bring = S1 * T_BYTES;          // the TMA ring starts at 0
-        sz = bring + S2 * BB_BYTES;
-        sfr = sz + BN * Gp * 4;
-        srs = sfr + 2 * BN * 4;
-        rflag = srs + BN * 4;
-        bars = rflag + 3 * 4 * 4;
-        tmem_slot = bars + (3 * MAX_S1 + 12) * 8;
+    int pring, rtile, rcur, rflag, bars, tmem_slot, abort, total;
+    __host__ __device__ SmemLayout(int XS, int CX, bool residual) {
+        pring = XS * CX * T_BYTES;  // the X ring starts at 0
+        rtile = pring + NPSLOT * PSLOT_BYTES;
+        rcur = rtile + (residual ? NSLOT * R_BYTES : 0);
+        rflag = rcur + (residual ? NSLOT * BN * 8 : 0);
+        bars = rflag + NSLOT * 4 * 4;
+        tmem_slot = bars + (2 * MAX_XS + 2 * NSLOT + 2 * NPSLOT + 8) * 8;
         abort = tmem_slot + 16;
-        col = abort + 16;
-        val = col + (csr_cap > 0 ? (csr_cap * 2 + 32 + 15) / 16 * 16 : 0);
-        total = val + (csr_cap > 0 ? (csr_cap / 2 + 32 + 15) / 16 * 16 : 0);
+        total = abort + 16;
     }
 };
-
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-                 : "memory");
-}
 
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols) {
@@ -128,13 +141,47 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
                             (static_cast<uint32_t>(BM >> 4) << 24);
 
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                        uint32_t accumulate) {
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major shared-memory tiles.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
         : "memory");
+}
+
+__device__ __forceinline__ void sts16(void *p, uint16_t v) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(smem_u32(p)), "h"(v) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T: A is M x 16 bf16 in tensor memory (lane =
+// row, two codes per 32-bit column), B an N x 16 K-major shared-memory tile.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 lanes x 32 columns of 32-bit values: thread i writes lane (base + i).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -160,81 +207,65 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// 32 lanes x 16 columns of 32-bit values: thread i gets lane (base + i).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-        "%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void sts128(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c),
-                 "r"(d)
-                 : "memory");
-}
-
-__device__ __forceinline__ void sts16(void *p, uint16_t v) {
-    asm volatile("st.shared.u16 [%0], %1;" ::"r"(smem_u32(p)), "h"(v) : "memory");
-}
-
 __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const SmemLayout L(p.S1, p.S2, p.Gp, p.csr_cap);
-    const int S1 = p.S1, S2 = p.S2;
+    const bool res = p.with_residual != 0;
+    const SmemLayout L(p.XS, p.CX, res);
+    const int XS = p.XS, CX = p.CX;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
     const int nk = p.K / BK;
     const int G = p.G, Gp = p.Gp;
+    // this CTA's tiles
+    const int t_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * p.tiles / gridDim.x);
+    const int t_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * p.tiles / gridDim.x);
 
-    const uint32_t *sz_s = reinterpret_cast<const uint32_t *>(smem + L.sz);
-    float *sfr = reinterpret_cast<float *>(smem + L.sfr);  // [2][BN] group scales
-    float *srs = reinterpret_cast<float *>(smem + L.srs);  // [BN] residual scales
-    volatile uint32_t *rflag = reinterpret_cast<volatile uint32_t *>(smem + L.rflag);  // [S2][4]
+    volatile uint32_t *rflag = reinterpret_cast<volatile uint32_t *>(smem + L.rflag);  // [NSLOT][4]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
-    uint64_t *full = bars;                 // [S1] TMA stage landed
-    uint64_t *empty = bars + MAX_S1;       // [S1] MMAs reading the TMA stage done
-    uint64_t *bready = bars + 2 * MAX_S1;  // [S2] operand buffer written
-    uint64_t *bempty = bready + 3;         // [S2] MMAs reading the operand buffer done
-    uint64_t *dfull = bready + 6;          // [2] group partial ready in TMEM
-    uint64_t *dempty = bready + 8;         // [2] epilogue done with the TMEM buffer
-    uint64_t *sready = bready + 10;        // [2] group scales written
-    uint64_t *rfull = bready + 12;         // residual accumulator complete
-    uint64_t *szbar = reinterpret_cast<uint64_t *>(smem + L.tmem_slot + 8);
+    uint64_t *full = bars;                 // [XS] X copy landed
+    uint64_t *empty = bars + MAX_XS;       // [XS] MMAs reading the X copy done
+    uint64_t *bready = bars + 2 * MAX_XS;  // [NSLOT] operand slot written
+    uint64_t *bempty = bready + NSLOT;     // [NSLOT] MMAs reading the operand slot done
+    uint64_t *dfull = bempty + NSLOT;      // [2] group partial ready in TMEM
+    uint64_t *dempty = dfull + 2;          // [2] epilogue done with the TMEM buffer
+    uint64_t *rfull = dempty + 2;          // every MMA of the tile complete
+    uint64_t *rempty = rfull + 1;          // epilogue done with the tile's R
+    uint64_t *pfull = rempty + 1;          // [NPSLOT] packed codes landed
+    uint64_t *pempty = pfull + NPSLOT;     // [NPSLOT] dequant done with the packed codes
+    const int spl = p.pw / 8;              // stages per packed-code load
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.tmem_slot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.abort);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S1; ++s) {
+        for (int s = 0; s < XS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < S2; ++b) {
+        for (int b = 0; b < NSLOT; ++b) {
             mbar_init(&bready[b], 4);
             mbar_init(&bempty[b], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&dfull[b], 1);
             mbar_init(&dempty[b], EPI_WARPS);
-            mbar_init(&sready[b], 4);
         }
         mbar_init(rfull, 1);
-        mbar_init(szbar, 1);
+        mbar_init(rempty, EPI_WARPS);
+        for (int b = 0; b < NPSLOT; ++b) {
+            mbar_init(&pfull[b], 1);
+            mbar_init(&pempty[b], 4);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (res) {
+        // the residual code tiles start zeroed; afterwards only written entries are cleared
+        for (int i = threadIdx.x; i < NSLOT * R_BYTES / 16; i += THREADS)
+            reinterpret_cast<uint4 *>(smem + L.rtile)[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async();
+    }
     if (warp == W_MMA) tmem_alloc(tmem_slot, TMEM_COLS);
-    for (int i = threadIdx.x; i < BN; i += THREADS)
-        srs[i] = (n0 + i < p.N) ? half_bits_to_f32(p.rscale[n0 + i]) : 0.f;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -245,220 +276,253 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
         if (lane == 0) {
             prefetch_tensormap(&p.tm_x);
             prefetch_tensormap(&p.tm_w);
-            prefetch_tensormap(&p.tm_sz);
-            mbar_arrive_expect_tx(szbar, BN * Gp * 4);
-            for (int j = 0; j < Gp / 4; ++j)
-                tma_load_2d(smem + L.sz + j * BN * 16, &p.tm_sz, szbar, 4 * j, n0);
-            int issued = 0;
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % S1;
-                if (i >= S1 &&
-                    !mbar_wait(&empty[s], ((i / S1) - 1) & 1, p.err, kErrWaitEmpty, abort_flag))
-                    break;
-                uint8_t *st = smem + s * T_BYTES;
-                mbar_arrive_expect_tx(&full[s], T_BYTES);
-                tma_load_2d(st, &p.tm_x, &full[s], i * BK, m0);
-                tma_load_2d(st + OFF_P, &p.tm_w, &full[s], i * (BK / 8), n0);
-                issued = i + 1;
+            int xc = 0, pc = 0;  // X and packed-code copies issued
+            bool ok = true;
+            for (int t = t_begin; ok && t < t_end; ++t) {
+                const int n0 = (t / p.m_tiles) * BN, m0 = (t % p.m_tiles) * BM;
+                for (int i = 0; i < nk; ++i) {
+                    if (i % spl == 0) {
+                        const int ps = pc % NPSLOT;
+                        if (pc >= NPSLOT && !mbar_wait(&pempty[ps], ((pc / NPSLOT) - 1) & 1, p.err,
+                                                       kErrWaitEmpty, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&pfull[ps], BN * p.pw * 4);
+                        tma_load_2d(smem + L.pring + ps * PSLOT_BYTES, &p.tm_w, &pfull[ps], i * (BK / 8), n0);
+                        ++pc;
+                    }
+                    if (i % CX == 0) {
+                        const int xs = xc % XS;
+                        if (xc >= XS &&
+                            !mbar_wait(&empty[xs], ((xc / XS) - 1) & 1, p.err, kErrWaitEmpty, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        // CX tiles; past the end of K the box reads zeros (and still
+                        // counts its full size)
+                        mbar_arrive_expect_tx(&full[xs], CX * T_BYTES);
+                        tma_load_3d(smem + xs * CX * T_BYTES, &p.tm_x, &full[xs], 0, m0, i);
+                        ++xc;
+                    }
+                }
             }
-            for (int i = max(0, issued - S1); i < issued; ++i)
-                mbar_wait(&full[i % S1], (i / S1) & 1, p.err, kErrWaitDrain, abort_flag);
-            mbar_wait(szbar, 0, p.err, kErrWaitDrain, abort_flag);
+            // no copy may still be in flight when the CTA exits
+            for (int j = max(0, xc - XS); j < xc; ++j)
+                mbar_wait(&full[j % XS], (j / XS) & 1, p.err, kErrWaitDrain, abort_flag);
+            for (int j = max(0, pc - NPSLOT); j < pc; ++j)
+                mbar_wait(&pfull[j % NPSLOT], (j / NPSLOT) & 1, p.err, kErrWaitDrain, abort_flag);
         }
     } else if (warp == W_MMA) {
         // ---------------------------------------------------------- MMA issue
         if (lane == 0) {
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % S1, g = i >> 1, b = g & 1, bb = i % S2;
-                if ((i & 1) == 0 && g >= 2 &&
-                    !mbar_wait(&dempty[b], ((g >> 1) - 1) & 1, p.err, kErrWaitMma, abort_flag))
-                    break;
-                if (!mbar_wait(&full[s], (i / S1) & 1, p.err, kErrWaitFull, abort_flag)) break;
-                if (!mbar_wait(&bready[bb], (i / S2) & 1, p.err, kErrWaitFull, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t bbuf = smem_u32(smem + L.bring + bb * BB_BYTES);
-                const uint64_t ad = sw128_desc(smem_u32(smem + s * T_BYTES));
-                const uint64_t bd = sw128_desc(bbuf);
-                const uint64_t br = sw128_desc(bbuf + B_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    mma_f16(tmem + b * BN, ad + 2 * kk, bd + 2 * kk, ((i & 1) | kk) ? 1u : 0u);
-                // stage 0 always runs, so the residual accumulator is initialized
-                if (p.with_residual &&
-                    (rflag[4 * bb] | rflag[4 * bb + 1] | rflag[4 * bb + 2] | rflag[4 * bb + 3])) {
+            int it = 0, gg0 = 0, xc = 0;
+            bool ok = true;
+            for (int t = t_begin, j = 0; ok && t < t_end; ++t, ++j, gg0 += G) {
+                for (int i = 0; i < nk; ++i, ++it) {
+                    const int xs = xc % XS, a = it % NSLOT;
+                    const int gg = gg0 + (i >> 1), b = gg & 1;
+                    if ((i & 1) == 0 && gg >= 2 &&
+                        !mbar_wait(&dempty[b], ((gg >> 1) - 1) & 1, p.err, kErrWaitMma, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if ((i % CX == 0 &&
+                         !mbar_wait(&full[xs], (xc / XS) & 1, p.err, kErrWaitFull, abort_flag)) ||
+                        !mbar_wait(&bready[a], (it / NSLOT) & 1, p.err, kErrWaitFull, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t xd = sw128_desc(smem_u32(smem + (xs * CX + i % CX) * T_BYTES));
+                    const uint32_t at = tmem + T_A + a * A_SLOT;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        mma_f16(tmem + 2 * BN, ad + 2 * kk, br + 2 * kk, (i | kk) ? 1u : 0u);
+                        mma_ts(tmem + T_D + b * BM, at + 8 * kk, xd + 2 * kk,
+                               ((i & 1) | kk) ? 1u : 0u);
+                    // stage 0 always runs, so R is initialized; it may be
+                    // overwritten once the epilogue has read the previous tile's R
+                    if (res && (rflag[4 * a] | rflag[4 * a + 1] | rflag[4 * a + 2] | rflag[4 * a + 3])) {
+                        if (i == 0 && j > 0 &&
+                            !mbar_wait(rempty, (j - 1) & 1, p.err, kErrWaitMma, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (i == 0) tc_fence_after();
+                        const uint64_t rd = sw128_desc(smem_u32(smem + L.rtile + a * R_BYTES));
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            mma_ss(tmem + T_R, rd + 2 * kk, xd + 2 * kk, (i | kk) ? 1u : 0u);
+                    }
+                    if (i % CX == CX - 1 || i == nk - 1) {
+                        mma_commit(&empty[xs]);
+                        ++xc;
+                    }
+                    mma_commit(&bempty[a]);
+                    if (i & 1) mma_commit(&dfull[b]);
                 }
-                mma_commit(&empty[s]);
-                mma_commit(&bempty[bb]);
-                if (i & 1) mma_commit(&dfull[b]);
+                // the epilogue waits for each tile's completion with the tile's parity,
+                // so it must have taken the previous one first
+                if (ok && !res && j > 0 &&
+                    !mbar_wait(rempty, (j - 1) & 1, p.err, kErrWaitMma, abort_flag))
+                    ok = false;
+                if (ok) mma_commit(rfull);
+                if (ok && t + 1 == t_end)  // every MMA has finished before TMEM is released
+                    mbar_wait(rfull, j & 1, p.err, kErrWaitDrain, abort_flag);
             }
-            mma_commit(rfull);
-            // every issued MMA has finished before tensor memory is released
-            mbar_wait(rfull, 0, p.err, kErrWaitDrain, abort_flag);
         }
     } else if (warp >= W_DQ0) {
         // ---------------------------------------------------------- dequant
-        const int n = (warp - W_DQ0) * 32 + lane;  // row within the tile
-        const int row = n0 + n;
-        const bool valid = row < p.N;
-        const bool res = p.with_residual != 0;
-        int cur = 0, end = 0;
-        const uint16_t *colp = p.col;  // residual columns, global or staged
-        const uint8_t *valp = p.val;
-        int cb = 0, vb = 0;            // index bases of the staged slice
-        if (res) {
-            if (valid) {
-                cur = p.row_ptr[row];
-                end = p.row_ptr[row + 1];
+        const int q = warp & 3;        // tensor-memory lane quadrant
+        const int n = 32 * q + lane;   // weight row within the tile (= lane)
+        const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16) + T_A;
+        int2 *rcur = reinterpret_cast<int2 *>(smem + L.rcur);  // [NSLOT][BN] entries written
+        int it = 0, pc = 0;
+        bool ok = true;
+        for (int t = t_begin; ok && t < t_end; ++t) {
+            const int row = (t / p.m_tiles) * BN + n;
+            const bool valid = row < p.N;
+            int cur = 0, end = 0;
+            if (res && valid) {
+                cur = __ldg(p.row_ptr + row);
+                end = __ldg(p.row_ptr + row + 1);
             }
-            if (p.csr_cap > 0) {
-                // stage this tile's CSR slice while the first TMA stages land
-                const int e_b = p.row_ptr[n0], e_e = p.row_ptr[min(n0 + BN, p.N)];
-                cb = e_b & ~7;
-                vb = (e_b >> 1) & ~15;
-                const int t = threadIdx.x - W_DQ0 * 32;
-                const int nc16 = (e_e > e_b) ? ((e_e - cb) * 2 + 15) / 16 : 0;
-                const int nv16 = (e_e > e_b) ? (((e_e + 1) >> 1) - vb + 15) / 16 : 0;
-                for (int k = t; k < nc16; k += 128) cp_async16(smem + L.col + 16 * k, p.col + cb + 8 * k);
-                for (int k = t; k < nv16; k += 128) cp_async16(smem + L.val + 16 * k, p.val + vb + 16 * k);
-                asm volatile("cp.async.wait_all;" ::: "memory");
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                colp = reinterpret_cast<const uint16_t *>(smem + L.col) - cb;
-                valp = smem + L.val - vb;
-            }
-        }
-        int nextc = (cur < end) ? static_cast<int>(colp[cur]) : 0x7fffffff;
-        uint32_t clean = 0;  // operand buffers whose residual rows of this warp are zero
-        bool ok = mbar_wait_warp(szbar, 0, p.err, kErrWaitFull, abort_flag);
-        for (int i = 0; ok && i < nk; ++i) {
-            const int s = i % S1, g = i >> 1, b = g & 1, bb = i % S2;
-            const uint32_t szw = sz_s[((g >> 2) * BN + n) * 4 + (g & 3)];
-            if ((i & 1) == 0) {
-                if (g >= 2 && !mbar_wait_warp(&dempty[b], ((g >> 1) - 1) & 1, p.err, kErrWaitMma,
-                                              abort_flag))
+            int nextc = (cur < end) ? static_cast<int>(__ldg(p.col + cur)) : 0x7fffffff;
+            for (int i = 0; i < nk; ++i, ++it) {
+                const int a = it % NSLOT, ps = pc % NPSLOT;
+                const uint32_t szw = valid ? __ldg(p.sz + static_cast<size_t>(row) * Gp + (i >> 1)) : 0u;
+                if ((i % spl == 0 &&
+                     !mbar_wait_warp(&pfull[ps], (pc / NPSLOT) & 1, p.err, kErrWaitFull, abort_flag)) ||
+                    (it >= NSLOT && !mbar_wait_warp(&bempty[a], ((it / NSLOT) - 1) & 1, p.err,
+                                                    kErrWaitMma, abort_flag))) {
+                    ok = false;
                     break;
-                sfr[b * BN + n] = half_bits_to_f32(szw);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sready[b]);
-            }
-            if (!mbar_wait_warp(&full[s], (i / S1) & 1, p.err, kErrWaitFull, abort_flag)) break;
-            if (i >= S2 &&
-                !mbar_wait_warp(&bempty[bb], ((i / S2) - 1) & 1, p.err, kErrWaitMma, abort_flag))
-                break;
-            uint8_t *st = smem + s * T_BYTES;
-            uint8_t *bbuf = smem + L.bring + bb * BB_BYTES;
-            const uint32_t z = static_cast<uint32_t>(half_bits_to_f32(szw >> 16));
-            const uint32_t zz = (0x4300u | z) * 0x00010001u;  // bf16x2 (128 + z)
-            const uint4 w0 = lds128(st + OFF_P + n * 32);
-            const uint4 w1 = lds128(st + OFF_P + n * 32 + 16);
-            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            uint8_t *brow = bbuf + n * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint32_t wd = words[c];
-                sts128(brow + ((c ^ (n & 7)) << 4), bf16x2_sub(nib_pair_bias128(wd), zz),
-                       bf16x2_sub(nib_pair_bias128(wd >> 4), zz),
-                       bf16x2_sub(nib_pair_bias128(wd >> 8), zz),
-                       bf16x2_sub(nib_pair_bias128(wd >> 12), zz));
-            }
-            bool has = false;
-            if (res) {
-                const int k_end = (i + 1) * BK;
-                has = __any_sync(0xffffffffu, nextc < k_end) || i == 0;
-                const uint32_t sbit = 1u << bb;
-                if (has || !(clean & sbit)) {
-                    uint8_t *rrow = bbuf + B_BYTES + n * 128;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) sts128(rrow + ((c ^ (n & 7)) << 4), 0u, 0u, 0u, 0u);
-                    while (nextc < k_end) {
-                        const int cl = nextc - i * BK;
-                        const uint32_t byte = valp[cur >> 1];
-                        const int qv = static_cast<int>(((byte >> ((cur & 1) * 4)) & 0xF) ^ 8) - 8;
-                        const __nv_bfloat16 qb = __float2bfloat16_rn(static_cast<float>(qv));
-                        sts16(rrow + (((cl >> 3) ^ (n & 7)) << 4) + (cl & 7) * 2,
-                              __bfloat16_as_ushort(qb));
-                        ++cur;
-                        nextc = (cur < end) ? static_cast<int>(colp[cur]) : 0x7fffffff;
-                    }
-                    clean = has ? (clean & ~sbit) : (clean | sbit);
                 }
+                tc_fence_after();
+                const uint32_t z = static_cast<uint32_t>(half_bits_to_f32(szw >> 16));
+                const uint32_t zz = (0x4300u | z) * 0x00010001u;  // bf16x2 (128 + z)
+                // this stage's two 16-byte chunks of the row (128-byte swizzle when pw = 32)
+                const uint8_t *prow = smem + L.pring + ps * PSLOT_BYTES + n * (p.pw * 4);
+                const int c0 = 2 * (i % spl), sw = (p.pw == 32) ? (n & 7) : 0;
+                const uint4 w0 = lds128(prow + ((c0 ^ sw) << 4));
+                const uint4 w1 = lds128(prow + (((c0 + 1) ^ sw) << 4));
+                if (i % spl == spl - 1 || i == nk - 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pempty[ps]);
+                    ++pc;
+                }
+                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                uint32_t codes[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    // pair j of word c holds columns (8c + 2j, 8c + 2j + 1)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        codes[4 * c + jj] = bf16x2_sub(nib_pair_bias128(words[c] >> (4 * jj)), zz);
+                }
+                tmem_st32(tl + a * A_SLOT, codes);
+                bool has = false;
+                if (res) {
+                    uint8_t *rrow = smem + L.rtile + a * R_BYTES + n * 128;
+                    const int sw = n & 7;
+                    if (it >= NSLOT) {
+                        // clear what this row wrote into the slot NSLOT stages ago
+                        const int2 wr = rcur[a * BN + n];
+                        const int k0o = ((it - NSLOT) % nk) * BK;
+                        for (int e = wr.x; e < wr.y; ++e) {
+                            const int cl = static_cast<int>(__ldg(p.col + e)) - k0o;
+                            sts16(rrow + (((cl >> 3) ^ sw) << 4) + (cl & 7) * 2, 0);
+                        }
+                    }
+                    const int k0 = i * BK, k_end = k0 + BK;
+                    const int first = cur;
+                    while (nextc < k_end) {
+                        const int cl = nextc - k0;
+                        const uint32_t byte = __ldg(p.val + (cur >> 1));
+                        const int qv = static_cast<int>(((byte >> ((cur & 1) * 4)) & 0xF) ^ 8) - 8;
+                        // q_r in [-8, 7] as bf16: exact
+                        sts16(rrow + (((cl >> 3) ^ sw) << 4) + (cl & 7) * 2,
+                              __bfloat16_as_ushort(__float2bfloat16_rn(static_cast<float>(qv))));
+                        ++cur;
+                        nextc = (cur < end) ? static_cast<int>(__ldg(p.col + cur)) : 0x7fffffff;
+                    }
+                    rcur[a * BN + n] = make_int2(first, cur);
+                    has = __any_sync(0xffffffffu, cur > first) || i == 0;
+                    fence_proxy_async();  // the tile is read by the tensor core
+                }
+                tmem_st_wait();
+                if (lane == 0) rflag[4 * a + q] = has ? 1u : 0u;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bready[a]);
             }
-            if (lane == 0) rflag[4 * bb + (warp - W_DQ0)] = has ? 1u : 0u;
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bready[bb]);
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        const int q = warp & 3;                        // tensor-memory lane quadrant
-        const int cb = ((warp - W_EPI0) >> 2) * EPI_COLS;  // first column of this warp
-        const int r = 32 * q + lane;                   // token within the tile
-        const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16) + cb;
-        float acc[EPI_COLS];
-#pragma unroll
-        for (int j = 0; j < EPI_COLS; ++j) acc[j] = 0.f;
+        const int q = warp & 3;                            // tensor-memory lane quadrant
+        const int tb = ((warp - W_EPI0) >> 2) * EPI_TOK;  // first token of this warp
+        const int n = 32 * q + lane;                       // weight row within the tile
+        const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16) + tb;
+        int gg = 0;
         bool ok = true;
-        for (int g = 0; g < G; ++g) {
-            const int b = g & 1;
-            if (!mbar_wait_warp(&dfull[b], (g >> 1) & 1, p.err, kErrWaitMma, abort_flag) ||
-                !mbar_wait_warp(&sready[b], (g >> 1) & 1, p.err, kErrWaitMma, abort_flag)) {
+        for (int t = t_begin, j = 0; ok && t < t_end; ++t, ++j) {
+            const int n0 = (t / p.m_tiles) * BN, m0 = (t % p.m_tiles) * BM;
+            const int row = n0 + n;
+            const bool valid = row < p.N;
+            float acc[EPI_TOK];
+#pragma unroll
+            for (int c = 0; c < EPI_TOK; ++c) acc[c] = 0.f;
+            for (int g = 0; g < G; ++g, ++gg) {
+                const int b = gg & 1;
+                const uint32_t szw = valid ? __ldg(p.sz + static_cast<size_t>(row) * Gp + g) : 0u;
+                if (!mbar_wait_warp(&dfull[b], (gg >> 1) & 1, p.err, kErrWaitMma, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float sc = half_bits_to_f32(szw & 0xFFFFu);
+#pragma unroll
+                for (int c0 = 0; c0 < EPI_TOK; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tl + T_D + b * BM + c0, v);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) acc[c0 + c] = fmaf(sc, v[c], acc[c0 + c]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dempty[b]);
+            }
+            if (!ok || !mbar_wait_warp(rfull, j & 1, p.err, kErrWaitMma, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const float *sc = sfr + b * BN + cb;
+            if (res) {
+                const float sr = valid ? half_bits_to_f32(__ldg(p.rscale + row)) : 0.f;
 #pragma unroll
-            for (int c0 = 0; c0 < EPI_COLS; c0 += 16) {
-                float v[16];
-                tmem_ld16(tl + b * BN + c0, v);
+                for (int c0 = 0; c0 < EPI_TOK; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tl + T_R + c0, v);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) acc[c0 + j] = fmaf(sc[c0 + j], v[j], acc[c0 + j]);
+                    for (int c = 0; c < 32; ++c) acc[c0 + c] = fmaf(sr, v[c], acc[c0 + c]);
+                }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&dempty[b]);
-        }
-        if (ok && mbar_wait_warp(rfull, 0, p.err, kErrWaitMma, abort_flag)) {
-            tc_fence_after();
-            if (p.with_residual) {
-#pragma unroll
-                for (int c0 = 0; c0 < EPI_COLS; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + 2 * BN + c0, v);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        acc[c0 + j] = fmaf(srs[cb + c0 + j], v[j], acc[c0 + j]);
-                }
-            }
-            const int tok = m0 + r;
-            const int nb = n0 + cb;
-            if (tok < p.M) {
+            if (lane == 0) mbar_arrive(rempty);
+            // a warp writes 32 consecutive outputs of one token per store
+            if (valid) {
+                const int nt = min(EPI_TOK, p.M - (m0 + tb));
                 if (p.Yf) {
-                    float *yr = p.Yf + static_cast<size_t>(tok) * p.N + nb;
+                    float *yc = p.Yf + static_cast<size_t>(m0 + tb) * p.N + row;
 #pragma unroll
-                    for (int j = 0; j < EPI_COLS; ++j)
-                        if (nb + j < p.N) yr[j] = acc[j];
+                    for (int c = 0; c < EPI_TOK; ++c)
+                        if (c < nt) yc[static_cast<size_t>(c) * p.N] = acc[c];
                 } else {
-                    __nv_bfloat16 *yr = p.Y + static_cast<size_t>(tok) * p.N + nb;
-                    if (nb + EPI_COLS <= p.N && (p.N & 7) == 0) {
+                    __nv_bfloat16 *yc = p.Y + static_cast<size_t>(m0 + tb) * p.N + row;
 #pragma unroll
-                        for (int j = 0; j < EPI_COLS; j += 8) {
-                            uint32_t pk[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                __nv_bfloat162 h =
-                                    __floats2bfloat162_rn(acc[j + 2 * e], acc[j + 2 * e + 1]);
-                                pk[e] = *reinterpret_cast<uint32_t *>(&h);
-                            }
-                            *reinterpret_cast<uint4 *>(yr + j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < EPI_COLS; ++j)
-                            if (nb + j < p.N) yr[j] = __float2bfloat16_rn(acc[j]);
-                    }
+                    for (int c = 0; c < EPI_TOK; ++c)
+                        if (c < nt) yc[static_cast<size_t>(c) * p.N] = __float2bfloat16_rn(acc[c]);
                 }
             }
         }
@@ -481,14 +545,19 @@ mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
     const PrefillMaps *pm = prefill_maps(w);
     if (!pm) return MQ_ERR_CUDA;
     PrefillParams p;
-    if (!encode_x_map(&p.tm_x, X, M, d.K))
+    p.with_residual = (partial == nullptr && d.nnz > 0) ? 1 : 0;
+    // four stages per X copy; two when the residual tiles take their share of
+    // shared memory (a deeper ring of smaller copies)
+    p.CX = p.with_residual ? 2 : 4;
+    if (!encode_x_map(&p.tm_x, X, M, d.K, p.CX))
         return fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for X");
     p.tm_w = pm->w;
-    p.tm_sz = pm->sz;
+    p.pw = pm->pw;
     p.row_ptr = d.row_ptr;
     p.col = d.col;
     p.val = d.val;
     p.rscale = d.rscale;
+    p.sz = d.sz;
     p.Y = static_cast<__nv_bfloat16 *>(Y);
     p.Yf = partial;
     p.err = d.err;
@@ -497,43 +566,32 @@ mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
     p.K = static_cast<int>(d.K);
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
-    p.with_residual = (partial == nullptr && d.nnz > 0) ? 1 : 0;
-    p.csr_cap = 0;
-    int cap = 0;
-    if (p.with_residual) {
-        const MapSet *ms = weight_maps(w, BN, 4);
-        if (!ms) return MQ_ERR_CUDA;
-        cap = static_cast<int>(ms->max_tile_nnz);
-    }
-    // deepest TMA ring that fits, keeping the residual slice in shared memory if possible
+    p.m_tiles = static_cast<int>((M + BM - 1) / BM);
+    const int64_t tiles = ((d.N + BN - 1) / BN) * static_cast<int64_t>(p.m_tiles);
+    if (tiles > (int64_t(1) << 30)) return fail(MQ_ERR_UNSUPPORTED, "prefill kernel: too many tiles");
+    p.tiles = static_cast<int>(tiles);
+    // the deepest X ring that fits
     const int budget = 227 * 1024 - 1024;
-    p.S1 = 0;
-    // prefer 3 operand buffers, then the deepest TMA ring (at least 4)
-    for (int s2 = 3; s2 >= 2 && !p.S1; --s2)
-        for (int s1 = MAX_S1; s1 >= (s2 == 3 ? 4 : 3) && !p.S1; --s1) {
-            if (SmemLayout(s1, s2, p.Gp, cap).total <= budget) {
-                p.S1 = s1;
-                p.S2 = s2;
-                p.csr_cap = cap;
-            } else if (s2 == 2 && s1 <= 4 && SmemLayout(s1, s2, p.Gp, 0).total <= budget) {
-                p.S1 = s1;
-                p.S2 = s2;
-            }
-        }
-    if (!p.S1) return fail(MQ_ERR_UNSUPPORTED, "prefill kernel: shared memory");
-    const SmemLayout L(p.S1, p.S2, p.Gp, p.csr_cap);
-    const int smem = L.total + 1024;
-    if (smem > 227 * 1024) return fail(MQ_ERR_UNSUPPORTED, "prefill kernel: shared memory");
+    p.XS = 0;
+    for (int xs = MAX_XS; xs >= 2 && !p.XS; --xs)
+        if (SmemLayout(xs, p.CX, p.with_residual != 0).total <= budget) p.XS = xs;
+    if (!p.XS) return fail(MQ_ERR_UNSUPPORTED, "prefill kernel: shared memory");
+    const int smem = SmemLayout(p.XS, p.CX, p.with_residual != 0).total + 1024;
     static bool configured[64] = {};
+    static int sms[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
+    if (dev < 0 || dev >= 64) return fail(MQ_ERR_UNSUPPORTED, "device ordinal above 63");
+    if (!configured[dev]) {
         if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 227 * 1024) != cudaSuccess)
-            return fail(MQ_ERR_CUDA, "cudaFuncSetAttribute failed for the prefill kernel");
+                                 227 * 1024) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            sms[dev] <= 0)
+            return fail(MQ_ERR_CUDA, "prefill kernel: device setup failed");
         configured[dev] = true;
     }
-    dim3 grid(static_cast<unsigned>((d.N + BN - 1) / BN), static_cast<unsigned>((M + BM - 1) / BM));
+    // one CTA per SM (its shared memory and 512 TMEM columns allow no second)
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, sms[dev]));
     prefill_kernel<<<grid, THREADS, smem, stream>>>(p);
     cudaError_t e = cudaPeekAtLastError();
     if (e != cudaSuccess)

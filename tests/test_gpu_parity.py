@@ -184,6 +184,7 @@ def test_prefill_full_size_sampled_rows(mq, cuda):
     (136, 11008, 40, 0.005),    # 86 groups (padded scale rows), ragged rows
     (300, 4096, 256, 0.01),     # two token tiles, three row tiles
     (128, 512, 17, 0.0),        # no residual
+    (130, 32768, 20, 0.002),    # longest K: scale/zero words read from global memory
 ])
 def test_prefill_kernel_shapes(mq, cuda, N, K, M, rho):
     W = synth.weight(N, K, std=0.02, outlier_frac=0.01, seed=N + K)
