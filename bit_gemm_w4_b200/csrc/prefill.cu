@@ -233,6 +233,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
     uint64_t *rempty = rfull + 1;          // epilogue done with the tile's R
     uint64_t *pfull = rempty + 1;          // [NPSLOT] packed codes landed
     uint64_t *pempty = pfull + NPSLOT;     // [NPSLOT] dequant done with the packed codes
+    static_assert(NSLOT == 4 && NPSLOT == 2, "slot arithmetic below uses shifts");
     const int spl = p.pw / 8;              // stages per packed-code load
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.tmem_slot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.abort);
@@ -273,17 +274,20 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
 
     if (warp == W_TMA) {
         // ---------------------------------------------------------- producer
+        // Slot indices and phases advance as counters: a lone thread would
+        // pay the full latency of every integer division by a runtime value.
         if (lane == 0) {
             prefetch_tensormap(&p.tm_x);
             prefetch_tensormap(&p.tm_w);
-            int xc = 0, pc = 0;  // X and packed-code copies issued
+            int xs = 0, xround = 0;  // X slot of the next copy, times the ring wrapped
+            int pc = 0, xc = 0;      // packed-code and X copies issued
             bool ok = true;
             for (int t = t_begin; ok && t < t_end; ++t) {
                 const int n0 = (t / p.m_tiles) * BN, m0 = (t % p.m_tiles) * BM;
-                for (int i = 0; i < nk; ++i) {
-                    if (i % spl == 0) {
-                        const int ps = pc % NPSLOT;
-                        if (pc >= NPSLOT && !mbar_wait(&pempty[ps], ((pc / NPSLOT) - 1) & 1, p.err,
+                for (int i = 0, pi = 0, xi = 0; i < nk; ++i) {
+                    if (pi == 0) {
+                        const int ps = pc & (NPSLOT - 1);
+                        if (pc >= NPSLOT && !mbar_wait(&pempty[ps], ((pc >> 1) - 1) & 1, p.err,
                                                        kErrWaitEmpty, abort_flag)) {
                             ok = false;
                             break;
@@ -292,49 +296,60 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                         tma_load_2d(smem + L.pring + ps * PSLOT_BYTES, &p.tm_w, &pfull[ps], i * (BK / 8), n0);
                         ++pc;
                     }
-                    if (i % CX == 0) {
-                        const int xs = xc % XS;
-                        if (xc >= XS &&
-                            !mbar_wait(&empty[xs], ((xc / XS) - 1) & 1, p.err, kErrWaitEmpty, abort_flag)) {
+                    if (++pi == spl) pi = 0;
+                    if (xi == 0) {
+                        if (xround > 0 &&
+                            !mbar_wait(&empty[xs], (xround - 1) & 1, p.err, kErrWaitEmpty, abort_flag)) {
                             ok = false;
                             break;
                         }
                         // CX tiles; past the end of K the box reads zeros (and still
                         // counts its full size)
                         mbar_arrive_expect_tx(&full[xs], CX * T_BYTES);
-                        tma_load_3d(smem + xs * CX * T_BYTES, &p.tm_x, &full[xs], 0, m0, i);
+                        tma_load_3d(smem + xs * (CX * T_BYTES), &p.tm_x, &full[xs], 0, m0, i);
                         ++xc;
+                        if (++xs == XS) {
+                            xs = 0;
+                            ++xround;
+                        }
                     }
+                    if (++xi == CX) xi = 0;
                 }
             }
-            // no copy may still be in flight when the CTA exits
-            for (int j = max(0, xc - XS); j < xc; ++j)
-                mbar_wait(&full[j % XS], (j / XS) & 1, p.err, kErrWaitDrain, abort_flag);
+            // no copy may still be in flight when the CTA exits: wait for the last
+            // XS X copies and the last two packed-code copies
+            for (int j = 0, s = xs, r = xround; j < XS && j < xc; ++j) {
+                if (--s < 0) {
+                    s = XS - 1;
+                    --r;
+                }
+                mbar_wait(&full[s], r & 1, p.err, kErrWaitDrain, abort_flag);
+            }
             for (int j = max(0, pc - NPSLOT); j < pc; ++j)
-                mbar_wait(&pfull[j % NPSLOT], (j / NPSLOT) & 1, p.err, kErrWaitDrain, abort_flag);
+                mbar_wait(&pfull[j & (NPSLOT - 1)], (j >> 1) & 1, p.err, kErrWaitDrain, abort_flag);
         }
     } else if (warp == W_MMA) {
         // ---------------------------------------------------------- MMA issue
         if (lane == 0) {
-            int it = 0, gg0 = 0, xc = 0;
+            int it = 0, gg0 = 0;
+            int xs = 0, xround = 0;  // X slot being read, times the ring wrapped
             bool ok = true;
             for (int t = t_begin, j = 0; ok && t < t_end; ++t, ++j, gg0 += G) {
-                for (int i = 0; i < nk; ++i, ++it) {
-                    const int xs = xc % XS, a = it % NSLOT;
+                for (int i = 0, xi = 0; i < nk; ++i, ++it) {
+                    const int a = it & (NSLOT - 1);
                     const int gg = gg0 + (i >> 1), b = gg & 1;
                     if ((i & 1) == 0 && gg >= 2 &&
                         !mbar_wait(&dempty[b], ((gg >> 1) - 1) & 1, p.err, kErrWaitMma, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    if ((i % CX == 0 &&
-                         !mbar_wait(&full[xs], (xc / XS) & 1, p.err, kErrWaitFull, abort_flag)) ||
-                        !mbar_wait(&bready[a], (it / NSLOT) & 1, p.err, kErrWaitFull, abort_flag)) {
+                    if ((xi == 0 && !mbar_wait(&full[xs], xround & 1, p.err, kErrWaitFull, abort_flag)) ||
+                        !mbar_wait(&bready[a], (it >> 2) & 1, p.err, kErrWaitFull, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t xd = sw128_desc(smem_u32(smem + (xs * CX + i % CX) * T_BYTES));
+                    const uint64_t xd = sw128_desc(smem_u32(smem + (xs * CX + xi) * T_BYTES));
                     const uint32_t at = tmem + T_A + a * A_SLOT;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
@@ -354,9 +369,13 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                         for (int kk = 0; kk < BK / 16; ++kk)
                             mma_ss(tmem + T_R, rd + 2 * kk, xd + 2 * kk, (i | kk) ? 1u : 0u);
                     }
-                    if (i % CX == CX - 1 || i == nk - 1) {
+                    if (++xi == CX || i == nk - 1) {
                         mma_commit(&empty[xs]);
-                        ++xc;
+                        xi = 0;
+                        if (++xs == XS) {
+                            xs = 0;
+                            ++xround;
+                        }
                     }
                     mma_commit(&bempty[a]);
                     if (i & 1) mma_commit(&dfull[b]);
@@ -378,6 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
         const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16) + T_A;
         int2 *rcur = reinterpret_cast<int2 *>(smem + L.rcur);  // [NSLOT][BN] entries written
         int it = 0, pc = 0;
+        int k0h[NSLOT] = {0, 0, 0, 0};  // first column of the last NSLOT stages (oldest last)
         bool ok = true;
         for (int t = t_begin; ok && t < t_end; ++t) {
             const int row = (t / p.m_tiles) * BN + n;
@@ -388,12 +408,13 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                 end = __ldg(p.row_ptr + row + 1);
             }
             int nextc = (cur < end) ? static_cast<int>(__ldg(p.col + cur)) : 0x7fffffff;
-            for (int i = 0; i < nk; ++i, ++it) {
-                const int a = it % NSLOT, ps = pc % NPSLOT;
-                const uint32_t szw = valid ? __ldg(p.sz + static_cast<size_t>(row) * Gp + (i >> 1)) : 0u;
-                if ((i % spl == 0 &&
-                     !mbar_wait_warp(&pfull[ps], (pc / NPSLOT) & 1, p.err, kErrWaitFull, abort_flag)) ||
-                    (it >= NSLOT && !mbar_wait_warp(&bempty[a], ((it / NSLOT) - 1) & 1, p.err,
+            const uint32_t *szrow = p.sz + static_cast<size_t>(row) * Gp;
+            for (int i = 0, pi = 0; i < nk; ++i, ++it) {
+                const int a = it & (NSLOT - 1), ps = pc & (NPSLOT - 1);
+                const uint32_t szw = valid ? __ldg(szrow + (i >> 1)) : 0u;
+                if ((pi == 0 &&
+                     !mbar_wait_warp(&pfull[ps], (pc >> 1) & 1, p.err, kErrWaitFull, abort_flag)) ||
+                    (it >= NSLOT && !mbar_wait_warp(&bempty[a], ((it >> 2) - 1) & 1, p.err,
                                                     kErrWaitMma, abort_flag))) {
                     ok = false;
                     break;
@@ -403,10 +424,11 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                 const uint32_t zz = (0x4300u | z) * 0x00010001u;  // bf16x2 (128 + z)
                 // this stage's two 16-byte chunks of the row (128-byte swizzle when pw = 32)
                 const uint8_t *prow = smem + L.pring + ps * PSLOT_BYTES + n * (p.pw * 4);
-                const int c0 = 2 * (i % spl), sw = (p.pw == 32) ? (n & 7) : 0;
+                const int c0 = 2 * pi, sw = (p.pw == 32) ? (n & 7) : 0;
                 const uint4 w0 = lds128(prow + ((c0 ^ sw) << 4));
                 const uint4 w1 = lds128(prow + (((c0 + 1) ^ sw) << 4));
-                if (i % spl == spl - 1 || i == nk - 1) {
+                if (++pi == spl || i == nk - 1) {
+                    pi = 0;
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pempty[ps]);
                     ++pc;
@@ -421,6 +443,11 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                         codes[4 * c + jj] = bf16x2_sub(nib_pair_bias128(words[c] >> (4 * jj)), zz);
                 }
                 tmem_st32(tl + a * A_SLOT, codes);
+                // k0h: first column of this stage and of the previous NSLOT - 1 stages
+                const int k0o = k0h[NSLOT - 1];
+#pragma unroll
+                for (int h = NSLOT - 1; h > 0; --h) k0h[h] = k0h[h - 1];
+                k0h[0] = i * BK;
                 bool has = false;
                 if (res) {
                     uint8_t *rrow = smem + L.rtile + a * R_BYTES + n * 128;
@@ -428,7 +455,6 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     if (it >= NSLOT) {
                         // clear what this row wrote into the slot NSLOT stages ago
                         const int2 wr = rcur[a * BN + n];
-                        const int k0o = ((it - NSLOT) % nk) * BK;
                         for (int e = wr.x; e < wr.y; ++e) {
                             const int cl = static_cast<int>(__ldg(p.col + e)) - k0o;
                             sts16(rrow + (((cl >> 3) ^ sw) << 4) + (cl & 7) * 2, 0);
