@@ -109,6 +109,31 @@ mq_status upload(mq_weight *w, T **dst, const T *src, size_t count, size_t pad_b
     return MQ_OK;
 }
 
+// The residual grouped per (128-row tile, 64-column stage, 32-row quadrant)
+// for the prefill kernel (layout in kernels.h, DeviceWeight::stage_ptr).
+void build_stage_lists(const HostPacked &hp, std::vector<int32_t> &ptr, std::vector<uint32_t> &ent) {
+    const int64_t tiles = (hp.N + 127) / 128, nk = hp.K / 64;
+    const int64_t keys = tiles * nk * 4;
+    ptr.assign(static_cast<size_t>(keys + 1), 0);
+    ent.assign(static_cast<size_t>(hp.nnz), 0u);
+    auto key = [&](int64_t n, int64_t c) { return ((n / 128) * nk + c / 64) * 4 + (n % 128) / 32; };
+    for (int64_t n = 0; n < hp.N; ++n)
+        for (int64_t e = hp.row_ptr[n]; e < hp.row_ptr[n + 1]; ++e) ++ptr[key(n, hp.col[e]) + 1];
+    for (int64_t k = 0; k < keys; ++k) ptr[k + 1] += ptr[k];
+    std::vector<int32_t> fill(ptr.begin(), ptr.end() - 1);
+    for (int64_t n = 0; n < hp.N; ++n)
+        for (int64_t e = hp.row_ptr[n]; e < hp.row_ptr[n + 1]; ++e) {
+            const int64_t c = hp.col[e];
+            const int q = static_cast<int>(((hp.val[e >> 1] >> ((e & 1) * 4)) & 0xF) ^ 8) - 8;
+            // q in [-8, 7] is exact in bf16: the high half of its fp32 bits
+            float f = static_cast<float>(q);
+            uint32_t bits;
+            std::memcpy(&bits, &f, 4);
+            ent[fill[key(n, c)]++] = static_cast<uint32_t>(n % 128) |
+                                     (static_cast<uint32_t>(c % 64) << 8) | (bits & 0xFFFF0000u);
+        }
+}
+
 mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **out) {
     *out = nullptr;
     int dev = -1;
@@ -136,6 +161,15 @@ mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **o
     if (!st) st = upload(w, &col, hp.col.data(), hp.col.size(), 64, stream);
     if (!st) st = upload(w, &val, hp.val.data(), hp.val.size(), 64, stream);
     if (!st) st = upload(w, &rs, hp.rscale.data(), hp.rscale.size(), 0, stream);
+    int32_t *sptr = nullptr;
+    uint32_t *sent = nullptr;
+    std::vector<int32_t> hptr;
+    std::vector<uint32_t> hent;
+    if (!st && hp.nnz > 0) {
+        build_stage_lists(hp, hptr, hent);
+        st = upload(w, &sptr, hptr.data(), hptr.size(), 0, stream);
+        if (!st) st = upload(w, &sent, hent.data(), hent.size(), 0, stream);
+    }
     if (!st) st = upload(w, &err, &zero, 1, 0, stream);
     if (!st) {
         e = cudaStreamSynchronize(stream);
@@ -151,6 +185,8 @@ mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **o
     d.col = col;
     d.val = val;
     d.rscale = rs;
+    d.stage_ptr = sptr;
+    d.stage_ent = sent;
     d.err = err;
     w->host_row_ptr = hp.row_ptr;
     for (int64_t n = 0; n < hp.N; ++n)

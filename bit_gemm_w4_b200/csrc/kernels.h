@@ -21,6 +21,13 @@ struct DeviceWeight {
     const uint16_t *col;      // [nnz] (+ padding)
     const uint8_t *val;       // [(nnz+1)/2] (+ padding)
     const uint16_t *rscale;   // [N]
+    // The residual again, grouped for the prefill kernel: per (128-row tile,
+    // 64-column stage, 32-row quadrant) the entries as words
+    // row-in-tile | column-in-stage << 8 | bf16 bits of q_r << 16, ordered by
+    // (tile, stage, quadrant, row, column); stage_ptr[(tile * K/64 + stage) * 4
+    // + quadrant] is the first entry of each group (one more entry at the end).
+    const int32_t *stage_ptr;   // [ceil(N/128) * K/64 * 4 + 1], NULL when nnz = 0
+    const uint32_t *stage_ent;  // [nnz]
     int *err;                 // device error word
 };
 

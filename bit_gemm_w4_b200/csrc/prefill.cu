@@ -76,9 +76,8 @@ static_assert(2 * T_BYTES >= BM * BN * 2, "the output tile is staged in the TMA 
 struct PrefillParams {
     CUtensorMap tm_x;  // X [M][K] bf16, box [128][64], 128B swizzle
     CUtensorMap tm_w;  // qweight [N][K/8] u32, box [128][8]
-    const int32_t *row_ptr;
-    const uint16_t *col;
-    const uint8_t *val;
+    const int32_t *stage_ptr;   // residual groups per (tile, stage, quadrant)
+    const uint32_t *stage_ent;
     const uint16_t *rscale;
     const uint32_t *sz;  // [N][Gp] scale | zero << 16
     __nv_bfloat16 *Y;
@@ -94,12 +93,11 @@ struct PrefillParams {
 };
 
 struct SmemLayout {
-    int pring, rtile, rcur, rflag, bars, tmem_slot, abort, total;
+    int pring, rtile, rflag, bars, tmem_slot, abort, total;
     __host__ __device__ SmemLayout(int XS, int CX, bool residual) {
         pring = XS * CX * T_BYTES;  // the X ring starts at 0
         rtile = pring + NPSLOT * PSLOT_BYTES;
-        rcur = rtile + (residual ? NSLOT * R_BYTES : 0);
-        rflag = rcur + (residual ? NSLOT * BN * 8 : 0);
+        rflag = rtile + (residual ? NSLOT * R_BYTES : 0);
         bars = rflag + NSLOT * 4 * 4;
         tmem_slot = bars + (2 * MAX_XS + 2 * NSLOT + 2 * NPSLOT + 8) * 8;
         abort = tmem_slot + 16;
@@ -225,8 +223,9 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *full = bars;                 // [XS] X copy landed
     uint64_t *empty = bars + MAX_XS;       // [XS] MMAs reading the X copy done
-    uint64_t *bready = bars + 2 * MAX_XS;  // [NSLOT] operand slot written
-    uint64_t *bempty = bready + NSLOT;     // [NSLOT] MMAs reading the operand slot done
+    // operand slots go back and forth in pairs (one 128-column group)
+    uint64_t *bready = bars + 2 * MAX_XS;  // [2] operand slot pair written
+    uint64_t *bempty = bready + NSLOT;     // [2] MMAs reading the slot pair done
     uint64_t *dfull = bempty + NSLOT;      // [2] group partial ready in TMEM
     uint64_t *dempty = dfull + 2;          // [2] epilogue done with the TMEM buffer
     uint64_t *rfull = dempty + 2;          // every MMA of the tile complete
@@ -243,7 +242,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < NSLOT; ++b) {
+        for (int b = 0; b < 2; ++b) {
             mbar_init(&bready[b], 4);
             mbar_init(&bempty[b], 1);
         }
@@ -335,41 +334,47 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
             int xs = 0, xround = 0;  // X slot being read, times the ring wrapped
             bool ok = true;
             for (int t = t_begin, j = 0; ok && t < t_end; ++t, ++j, gg0 += G) {
-                for (int i = 0, xi = 0; i < nk; ++i, ++it) {
-                    const int a = it & (NSLOT - 1);
-                    const int gg = gg0 + (i >> 1), b = gg & 1;
-                    if ((i & 1) == 0 && gg >= 2 &&
+                // two stages (one group, one operand slot pair) per step
+                for (int i = 0, xi = 0; i < nk; i += 2, it += 2) {
+                    const int gg = gg0 + (i >> 1), b = gg & 1, pp = (it >> 1) & 1;
+                    if (gg >= 2 &&
                         !mbar_wait(&dempty[b], ((gg >> 1) - 1) & 1, p.err, kErrWaitMma, abort_flag)) {
                         ok = false;
                         break;
                     }
                     if ((xi == 0 && !mbar_wait(&full[xs], xround & 1, p.err, kErrWaitFull, abort_flag)) ||
-                        !mbar_wait(&bready[a], (it >> 2) & 1, p.err, kErrWaitFull, abort_flag)) {
+                        !mbar_wait(&bready[pp], (it >> 2) & 1, p.err, kErrWaitFull, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t xd = sw128_desc(smem_u32(smem + (xs * CX + xi) * T_BYTES));
-                    const uint32_t at = tmem + T_A + a * A_SLOT;
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        mma_ts(tmem + T_D + b * BM, at + 8 * kk, xd + 2 * kk,
-                               ((i & 1) | kk) ? 1u : 0u);
-                    // stage 0 always runs, so R is initialized; it may be
-                    // overwritten once the epilogue has read the previous tile's R
-                    if (res && (rflag[4 * a] | rflag[4 * a + 1] | rflag[4 * a + 2] | rflag[4 * a + 3])) {
-                        if (i == 0 && j > 0 &&
-                            !mbar_wait(rempty, (j - 1) & 1, p.err, kErrWaitMma, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        if (i == 0) tc_fence_after();
-                        const uint64_t rd = sw128_desc(smem_u32(smem + L.rtile + a * R_BYTES));
+                    for (int h = 0; h < 2; ++h) {
+                        const int a = (it + h) & (NSLOT - 1);
+                        const uint64_t xd = sw128_desc(smem_u32(smem + (xs * CX + xi + h) * T_BYTES));
+                        const uint32_t at = tmem + T_A + a * A_SLOT;
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
-                            mma_ss(tmem + T_R, rd + 2 * kk, xd + 2 * kk, (i | kk) ? 1u : 0u);
+                            mma_ts(tmem + T_D + b * BM, at + 8 * kk, xd + 2 * kk, (h | kk) ? 1u : 0u);
+                        // stage 0 always runs, so R is initialized; it may be
+                        // overwritten once the epilogue has read the previous tile's R
+                        if (res && (rflag[4 * a] | rflag[4 * a + 1] | rflag[4 * a + 2] | rflag[4 * a + 3])) {
+                            if (i + h == 0 && j > 0) {
+                                if (!mbar_wait(rempty, (j - 1) & 1, p.err, kErrWaitMma, abort_flag)) {
+                                    ok = false;
+                                    break;
+                                }
+                                tc_fence_after();
+                            }
+                            const uint64_t rd = sw128_desc(smem_u32(smem + L.rtile + a * R_BYTES));
+#pragma unroll
+                            for (int kk = 0; kk < BK / 16; ++kk)
+                                mma_ss(tmem + T_R, rd + 2 * kk, xd + 2 * kk, ((i + h) | kk) ? 1u : 0u);
+                        }
                     }
-                    if (++xi == CX || i == nk - 1) {
+                    if (!ok) break;
+                    xi += 2;
+                    if (xi == CX || i + 2 == nk) {
                         mma_commit(&empty[xs]);
                         xi = 0;
                         if (++xs == XS) {
@@ -377,8 +382,8 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                             ++xround;
                         }
                     }
-                    mma_commit(&bempty[a]);
-                    if (i & 1) mma_commit(&dfull[b]);
+                    mma_commit(&bempty[pp]);
+                    mma_commit(&dfull[b]);
                 }
                 // the epilogue waits for each tile's completion with the tile's parity,
                 // so it must have taken the previous one first
@@ -395,27 +400,28 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
         const int q = warp & 3;        // tensor-memory lane quadrant
         const int n = 32 * q + lane;   // weight row within the tile (= lane)
         const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16) + T_A;
-        int2 *rcur = reinterpret_cast<int2 *>(smem + L.rcur);  // [NSLOT][BN] entries written
         int it = 0, pc = 0;
-        int k0h[NSLOT] = {0, 0, 0, 0};  // first column of the last NSLOT stages (oldest last)
+        // the residual groups this warp wrote in the last NSLOT stages (oldest last)
+        int h0[NSLOT] = {0, 0, 0, 0}, h1[NSLOT] = {0, 0, 0, 0};
         bool ok = true;
         for (int t = t_begin; ok && t < t_end; ++t) {
             const int row = (t / p.m_tiles) * BN + n;
             const bool valid = row < p.N;
-            int cur = 0, end = 0;
-            if (res && valid) {
-                cur = __ldg(p.row_ptr + row);
-                end = __ldg(p.row_ptr + row + 1);
-            }
-            int nextc = (cur < end) ? static_cast<int>(__ldg(p.col + cur)) : 0x7fffffff;
             const uint32_t *szrow = p.sz + static_cast<size_t>(row) * Gp;
+            const int32_t *gptr = res ? p.stage_ptr + (static_cast<size_t>(t / p.m_tiles) * nk) * 4 + q : nullptr;
             for (int i = 0, pi = 0; i < nk; ++i, ++it) {
                 const int a = it & (NSLOT - 1), ps = pc & (NPSLOT - 1);
                 const uint32_t szw = valid ? __ldg(szrow + (i >> 1)) : 0u;
+                int g0 = 0, g1 = 0;  // this warp's residual group of the stage
+                if (res) {
+                    g0 = __ldg(gptr + 4 * i);
+                    g1 = __ldg(gptr + 4 * i + 1);
+                }
                 if ((pi == 0 &&
                      !mbar_wait_warp(&pfull[ps], (pc >> 1) & 1, p.err, kErrWaitFull, abort_flag)) ||
-                    (it >= NSLOT && !mbar_wait_warp(&bempty[a], ((it >> 2) - 1) & 1, p.err,
-                                                    kErrWaitMma, abort_flag))) {
+                    ((it & 1) == 0 && it >= NSLOT &&
+                     !mbar_wait_warp(&bempty[(it >> 1) & 1], ((it >> 2) - 1) & 1, p.err, kErrWaitMma,
+                                     abort_flag))) {
                     ok = false;
                     break;
                 }
@@ -443,44 +449,44 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                         codes[4 * c + jj] = bf16x2_sub(nib_pair_bias128(words[c] >> (4 * jj)), zz);
                 }
                 tmem_st32(tl + a * A_SLOT, codes);
-                // k0h: first column of this stage and of the previous NSLOT - 1 stages
-                const int k0o = k0h[NSLOT - 1];
-#pragma unroll
-                for (int h = NSLOT - 1; h > 0; --h) k0h[h] = k0h[h - 1];
-                k0h[0] = i * BK;
                 bool has = false;
                 if (res) {
-                    uint8_t *rrow = smem + L.rtile + a * R_BYTES + n * 128;
-                    const int sw = n & 7;
-                    if (it >= NSLOT) {
-                        // clear what this row wrote into the slot NSLOT stages ago
-                        const int2 wr = rcur[a * BN + n];
-                        for (int e = wr.x; e < wr.y; ++e) {
-                            const int cl = static_cast<int>(__ldg(p.col + e)) - k0o;
-                            sts16(rrow + (((cl >> 3) ^ sw) << 4) + (cl & 7) * 2, 0);
+                    uint8_t *rt = smem + L.rtile + a * R_BYTES;
+                    // clear this warp's entries of the stage that used the slot
+                    // NSLOT stages ago, then write the stage's entries; an entry
+                    // word holds row, column and the bf16 code ready to store
+                    const int o0 = h0[NSLOT - 1], o1 = h1[NSLOT - 1];
+#pragma unroll
+                    for (int h = NSLOT - 1; h > 0; --h) {
+                        h0[h] = h0[h - 1];
+                        h1[h] = h1[h - 1];
+                    }
+                    h0[0] = g0;
+                    h1[0] = g1;
+                    if (it >= NSLOT)
+                        for (int e = o0 + lane; e < o1; e += 32) {
+                            const uint32_t v = __ldg(p.stage_ent + e);
+                            const int r = v & 127, c = (v >> 8) & 63;
+                            sts16(rt + r * 128 + (((c >> 3) ^ (r & 7)) << 4) + (c & 7) * 2, 0);
                         }
+                    __syncwarp();
+                    for (int e = g0 + lane; e < g1; e += 32) {
+                        const uint32_t v = __ldg(p.stage_ent + e);
+                        const int r = v & 127, c = (v >> 8) & 63;
+                        sts16(rt + r * 128 + (((c >> 3) ^ (r & 7)) << 4) + (c & 7) * 2,
+                              static_cast<uint16_t>(v >> 16));
                     }
-                    const int k0 = i * BK, k_end = k0 + BK;
-                    const int first = cur;
-                    while (nextc < k_end) {
-                        const int cl = nextc - k0;
-                        const uint32_t byte = __ldg(p.val + (cur >> 1));
-                        const int qv = static_cast<int>(((byte >> ((cur & 1) * 4)) & 0xF) ^ 8) - 8;
-                        // q_r in [-8, 7] as bf16: exact
-                        sts16(rrow + (((cl >> 3) ^ sw) << 4) + (cl & 7) * 2,
-                              __bfloat16_as_ushort(__float2bfloat16_rn(static_cast<float>(qv))));
-                        ++cur;
-                        nextc = (cur < end) ? static_cast<int>(__ldg(p.col + cur)) : 0x7fffffff;
-                    }
-                    rcur[a * BN + n] = make_int2(first, cur);
-                    has = __any_sync(0xffffffffu, cur > first) || i == 0;
+                    // stage 0 of a tile always runs its residual MMAs (R starts there)
+                    has = g1 > g0 || i == 0;
                     fence_proxy_async();  // the tile is read by the tensor core
                 }
                 tmem_st_wait();
                 if (lane == 0) rflag[4 * a + q] = has ? 1u : 0u;
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bready[a]);
+                if (it & 1) {  // the pair's second stage: hand the pair over
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bready[(it >> 1) & 1]);
+                }
             }
         }
     } else {
@@ -579,9 +585,8 @@ mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
         return fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for X");
     p.tm_w = pm->w;
     p.pw = pm->pw;
-    p.row_ptr = d.row_ptr;
-    p.col = d.col;
-    p.val = d.val;
+    p.stage_ptr = d.stage_ptr;
+    p.stage_ent = d.stage_ent;
     p.rscale = d.rscale;
     p.sz = d.sz;
     p.Y = static_cast<__nv_bfloat16 *>(Y);
