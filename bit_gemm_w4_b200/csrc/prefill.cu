@@ -480,9 +480,9 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     has = g1 > g0 || i == 0;
                     fence_proxy_async();  // the tile is read by the tensor core
                 }
-                tmem_st_wait();
                 if (lane == 0) rflag[4 * a + q] = has ? 1u : 0u;
                 if (it & 1) {  // the pair's second stage: hand the pair over
+                    tmem_st_wait();  // both stages' codes are in tensor memory
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bready[(it >> 1) & 1]);
