@@ -16,6 +16,9 @@ is no data-path collective. Rank 0 prints one JSON line.
 Also reported (secondary): the 70B-MLP batched decode (M = 16) in TB/s and
 the prefill (M = 2048) in TFLOP/s, each with its roofline fraction.
 
+python bench.py --profile-case NAME [--reps R] runs one small case of the hot
+path a few times and prints its launch time (the command ncu captures use).
+
 --impl reference times the fp64 CPU oracle on a bounded row sample of the
 same workload (rank 0 only) and prints the same JSON line with
 "impl": "reference".
@@ -56,6 +59,14 @@ def alg_bytes(M: int, N: int, K: int, nnz: int) -> int:
     (row_ptr, col, val, rscale), X and Y, each once."""
     return (N * K // 2 + 4 * N * (K // 128) + 4 * (N + 1) + 2 * nnz + (nnz + 1) // 2 + 2 * N
             + 2 * M * K + 2 * M * N)
+
+
+# DRAM bytes (read + write) of one decode launch, 4096 x 4096, M = 1, density
+# 0.5 %, from one ncu capture of the current decode kernel (the summary under
+# profiles/ gives the command). The bench's other shapes are scaled by their
+# packed size N*K, which the traffic follows (no re-reads). Set to None when
+# the decode kernel changes until it is captured again.
+DECODE_TRAFFIC_4096 = 9.198592e6
 
 
 def alg_flops(M: int, N: int, K: int, nnz: int) -> int:
@@ -362,7 +373,12 @@ def run_ours(args):
                          f"({copies * step_bytes / 1e6:.0f} MB) vs L2 {l2 / 1e6:.0f} MB",
                    "parallelism": f"replicas x{dist_ctx.world}", "timing": "CUDA graph replay"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
-                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+                     "traffic": (None if DECODE_TRAFFIC_4096 is None else
+                                 round(sum(DECODE_TRAFFIC_4096 * N * K / 4096 ** 2
+                                           for N, K in ds.shapes))),
+                     "traffic_note": "DRAM bytes per step (3 launches): one ncu capture of the "
+                                     "4096x4096 launch scaled by N*K",
                      "peak_source": pk_src,
                      "kernel": "decode_kernel (the step's three launches)",
                      "per_shape_us": {f"{N}x{K}": round(t * 1e3, 3)
@@ -456,8 +472,54 @@ def run_reference(args):
     }), flush=True)
 
 
+# ------------------------------------------------------------------ profile cases
+PROFILE_CASES = {
+    # name: (N, K, M, rho, path)
+    "decode-4096x4096-m1": (4096, 4096, 1, 0.005, "auto"),
+    "decode-11008x4096-m1": (11008, 4096, 1, 0.005, "auto"),
+    "decode-28672x8192-m16": (28672, 8192, 16, 0.01, "auto"),
+    "prefill-14336x4096-m256": (14336, 4096, 256, 0.005, "prefill"),
+    "prefill-14336x4096-m2048": (14336, 4096, 2048, 0.005, "prefill"),
+}
+
+
+def run_profile_case(name: str, reps: int):
+    """One small case of the hot path, a few timed launches (CUDA events,
+    L2 flushed before each): the command the ncu summaries are taken with.
+    Prints one JSON line with the median launch time; not a bench line."""
+    import torch
+    from bit_gemm_w4_b200 import mosaicq as mq, synth
+    N, K, M, rho, path = PROFILE_CASES[name]
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=1)
+    w = mq.Weight.pack(W, rho)
+    X = synth.activations(M, K, seed=2, channels=8, mult=30.0).to(dev)
+    Y = w.linear(X, path=path)
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        w.linear(X, Y, path=path)
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    if w.device_error() != 0:
+        raise RuntimeError("device error word set")
+    nnz = w.info()["nnz"]
+    t = statistics.median(ts)
+    print(json.dumps({"profile_case": name, "N": N, "K": K, "M": M, "rho": rho, "path": path,
+                      "us": round(t, 2), "TB_s": round(alg_bytes(M, N, K, nnz) / t / 1e6, 3),
+                      "TFLOP_s": round(alg_flops(M, N, K, nnz) / t / 1e6, 1)}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run one small case a few times (the ncu capture command) and exit")
+    ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
@@ -466,6 +528,9 @@ def main(argv=None):
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args(argv)
+    if args.profile_case:
+        run_profile_case(args.profile_case, args.reps)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
