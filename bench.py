@@ -16,6 +16,9 @@ is no data-path collective. Rank 0 prints one JSON line.
 Also reported (secondary): the 70B-MLP batched decode (M = 16) in TB/s and
 the prefill (M = 2048) in TFLOP/s, each with its roofline fraction.
 
+python bench.py --overhead [--reps R] measures the residual's cost, fused and
+unfused, against density 0.
+
 python bench.py --profile-case NAME [--reps R] runs one small case of the hot
 path a few times and prints its launch time (the command ncu captures use).
 
@@ -515,11 +518,68 @@ def run_profile_case(name: str, reps: int):
                       "TFLOP_s": round(alg_flops(M, N, K, nnz) / t / 1e6, 1)}))
 
 
+# ------------------------------------------------------------------ residual overhead
+def run_overhead(reps: int):
+    """The cost of the residual, fused and unfused: each shape packed at
+    several densities from the same weight; every launch timed with CUDA
+    events after an L2 flush (median of reps). Reports, per shape and density,
+    the fused time, the unfused (dense kernel + separate residual kernel) time
+    and the fused overhead over density 0 (MosaicQuant, "Experimental Results":
+    the fused sparse branches' latency overhead). Prints one JSON line."""
+    import torch
+    from bit_gemm_w4_b200 import mosaicq as mq, synth
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    cases = [("qkvo", 4096, 4096, 1), ("gateup", 11008, 4096, 1), ("down", 4096, 11008, 1),
+             ("qkvo", 4096, 4096, 16), ("prefill", 14336, 4096, 2048)]
+    rhos = (0.0, 0.0025, 0.005, 0.01, 0.04)
+
+    def timed(fn):
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        return statistics.median(ts)
+
+    rows = []
+    for name, N, K, M in cases:
+        W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=1)
+        X = synth.activations(M, K, seed=2, channels=8, mult=30.0).to(dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty((M, N), dtype=torch.float32, device=dev)
+        base = None
+        for rho in rhos:
+            w = mq.Weight.pack(W, rho)
+            w.linear(X, Y)
+            w.linear_unfused(X, Y, ws)
+            torch.cuda.synchronize()
+            fused = timed(lambda: w.linear(X, Y))
+            unfused = timed(lambda: w.linear_unfused(X, Y, ws))
+            if w.device_error() != 0:
+                raise RuntimeError("device error word set")
+            base = fused if rho == 0.0 else base
+            rows.append({"shape": name, "N": N, "K": K, "M": M, "rho": rho,
+                         "nnz": w.info()["nnz"], "fused_us": round(fused, 2),
+                         "unfused_us": round(unfused, 2),
+                         "fused_overhead_vs_rho0": round(fused / base - 1.0, 4),
+                         "unfused_over_fused": round(unfused / fused, 3)})
+            w.free()
+    print(json.dumps({"overhead": rows, "timing": f"CUDA events, L2 flushed, median of {reps}"}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
                     help="run one small case a few times (the ncu capture command) and exit")
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--overhead", action="store_true",
+                    help="measure the residual's fused and unfused overhead over density 0 and exit")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
@@ -530,6 +590,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.profile_case:
         run_profile_case(args.profile_case, args.reps)
+        return
+    if args.overhead:
+        run_overhead(max(args.reps, 5))
         return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
