@@ -203,3 +203,40 @@ def test_prefill_kernel_dense_residual(mq, cuda):
     assert w.device_error() == 0
     r = oracle_check(Y, X, oracle.from_arrays(dd))
     assert r["ok"], r
+
+
+def _row_subset(dd: dict, rows: np.ndarray) -> dict:
+    """The decomposition restricted to the given rows (arrays re-indexed)."""
+    rp = np.asarray(dd["row_ptr"], np.int64)
+    idx = np.concatenate([np.arange(rp[r], rp[r + 1]) for r in rows]) if len(rows) else np.zeros(0, np.int64)
+    counts = rp[rows + 1] - rp[rows]
+    return dict(N=len(rows), K=dd["K"], q=dd["q"][rows], s=dd["s"][rows], z=dd["z"][rows],
+                row_ptr=np.concatenate([[0], np.cumsum(counts)]).astype(np.int64),
+                col=np.asarray(dd["col"])[idx], qr=np.asarray(dd["qr"])[idx], sr=dd["sr"][rows])
+
+
+@pytest.mark.parametrize("rho", synth.SWEEP_RHO)
+@pytest.mark.parametrize("shape", sorted(synth.SWEEP_SHAPES))
+def test_sweep_grid(mq, cuda, shape, rho):
+    """The density sweep: Llama-7B block linears at every M of the sweep
+    (decode and prefill kernels) and every density, on clustered synthetic
+    decompositions; packed rows byte-exact and outputs within the bounds on
+    48 sampled rows (first, last and random)."""
+    N, K = synth.SWEEP_SHAPES[shape]
+    k_n = int(np.floor(rho * K + 0.5))
+    dd = synth.sweep_decomposition(N, K, k_n, seed=N + K + k_n)
+    w = mq.Weight.pack_decomposed(dd)
+    rows = np.unique(np.concatenate([np.arange(0, 16), np.arange(N - 16, N),
+                                     np.random.default_rng(k_n).choice(N, 16, replace=False)]))
+    sub = _row_subset(dd, rows)
+    d = oracle.from_arrays(sub)
+    ex, want = w.export(), oracle.pack(d)
+    for key in ("qweight", "sz", "rscale"):
+        assert np.array_equal(ex[key][rows], want[key]), key
+    for M in synth.SWEEP_M:
+        X = synth.activations(M, K, seed=M + k_n)
+        Y = w.linear(X.cuda())
+        torch.cuda.synchronize()
+        assert w.device_error() == 0
+        r = oracle_check(Y[:, rows], X, d)
+        assert r["ok"], (M, r)
