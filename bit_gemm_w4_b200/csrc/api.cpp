@@ -288,7 +288,9 @@ const char *mq_last_error(void) { return g_last_error.c_str(); }
 mq_status mq_residual_nnz(int64_t N, int64_t K, const mq_pack_opts *opts, int64_t *nnz) {
     if (!nnz) return fail(MQ_ERR_INVALID_ARG, "nnz is NULL");
     if (mq_status st = check_shape(N, K, opts)) return st;
-    *nnz = N * residual_count(K, opts->residual_density);
+    *nnz = opts->residual_blocks == 1
+               ? residual_blocks_selected(N, K, opts->block_fraction) * kBlockRows * kBlockCols
+               : N * residual_count(K, opts->residual_density);
     return MQ_OK;
 }
 
@@ -299,7 +301,7 @@ mq_status mq_pack_host(const float *W_host, int64_t N, int64_t K, const mq_pack_
     if (!out->qweight || !out->sz || !out->row_ptr || !out->rscale)
         return fail(MQ_ERR_INVALID_ARG, "an output buffer is NULL");
     HostDecomp d;
-    if (mq_status st = decompose_host(W_host, N, K, opts->residual_density, d)) return st;
+    if (mq_status st = decompose_host(W_host, N, K, *opts, d)) return st;
     if (!d.col.empty() && (!out->col || !out->val))
         return fail(MQ_ERR_INVALID_ARG, "col/val buffers are NULL");
     HostPacked p;
@@ -323,7 +325,7 @@ mq_status mq_pack(const float *W_host, int64_t N, int64_t K, const mq_pack_opts 
     if (!W_host) return fail(MQ_ERR_INVALID_ARG, "W is NULL");
     if (mq_status st = check_shape(N, K, opts)) return st;
     HostDecomp d;
-    if (mq_status st = decompose_host(W_host, N, K, opts->residual_density, d)) return st;
+    if (mq_status st = decompose_host(W_host, N, K, *opts, d)) return st;
     HostPacked p;
     try {
         pack_host(view_of(d), p);

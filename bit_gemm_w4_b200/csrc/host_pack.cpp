@@ -73,10 +73,29 @@ mq_status check_shape(int64_t N, int64_t K, const mq_pack_opts *opts) {
     if (K % kGroup) return fail(MQ_ERR_INVALID_ARG, "K must be a multiple of 128");
     if (K > 65536) return fail(MQ_ERR_INVALID_ARG, "K must be at most 65536 (u16 columns)");
     if (N > (int64_t(1) << 31) - 1) return fail(MQ_ERR_INVALID_ARG, "N too large");
-    double rho = opts->residual_density;
-    if (!(rho >= 0.0 && rho <= 1.0))
-        return fail(MQ_ERR_INVALID_ARG, "residual_density must be in [0, 1]");
+    if (opts->residual_blocks == 0) {
+        double rho = opts->residual_density;
+        if (!(rho >= 0.0 && rho <= 1.0))
+            return fail(MQ_ERR_INVALID_ARG, "residual_density must be in [0, 1]");
+    } else if (opts->residual_blocks == 1) {
+        double f = opts->block_fraction;
+        if (!(f >= 0.0 && f <= 1.0)) return fail(MQ_ERR_INVALID_ARG, "block_fraction must be in [0, 1]");
+        if (N % kBlockRows) return fail(MQ_ERR_INVALID_ARG, "block mode needs N % 16 == 0");
+        if (opts->channel_weight)
+            for (int64_t k = 0; k < K; ++k) {
+                const double h = opts->channel_weight[k];
+                if (!(std::isfinite(h) && h >= 0.0))
+                    return fail(MQ_ERR_INVALID_ARG, "channel weights must be finite and >= 0");
+            }
+    } else {
+        return fail(MQ_ERR_UNSUPPORTED, "unknown residual_blocks mode");
+    }
     return MQ_OK;
+}
+
+int64_t residual_blocks_selected(int64_t N, int64_t K, double fraction) {
+    const int64_t blocks = (N / kBlockRows) * (K / kBlockCols);
+    return static_cast<int64_t>(std::floor(fraction * static_cast<double>(blocks) + 0.5));
 }
 
 namespace {
@@ -86,13 +105,11 @@ struct RowError {
     std::string msg;
 };
 
-// Decompose rows [r0, r1) of W into d (already sized).
-void decompose_rows(const float *W, int64_t K, int64_t k_n, int64_t r0, int64_t r1,
-                    HostDecomp &d, RowError &err) {
+// D1 and D2 for row n: codes, scales and zero points into d, the errors
+// E = w - deq into E[0..K). Returns false (with err set) on bad input.
+bool base_row(const float *W, int64_t K, int64_t n, HostDecomp &d, double *E, RowError &err) {
     const int64_t G = K / kGroup;
-    std::vector<double> E(K), absE(K);
-    std::vector<int32_t> idx(K);
-    for (int64_t n = r0; n < r1; ++n) {
+    {
         const float *w = W + n * K;
         uint8_t *q = d.q.data() + n * K;
         for (int64_t g = 0; g < G; ++g) {
@@ -103,7 +120,7 @@ void decompose_rows(const float *W, int64_t K, int64_t k_n, int64_t r0, int64_t 
                 if (!std::isfinite(x)) {
                     err.bad = true;
                     err.msg = "W holds NaN or Inf";
-                    return;
+                    return false;
                 }
                 lo = std::min(lo, x);
                 hi = std::max(hi, x);
@@ -112,7 +129,7 @@ void decompose_rows(const float *W, int64_t K, int64_t k_n, int64_t r0, int64_t 
             if ((sb & 0x7FFF) == 0x7C00) {
                 err.bad = true;
                 err.msg = "a group scale overflows fp16";
-                return;
+                return false;
             }
             if (hi == lo)
                 sb = 0x3C00;  // 1.0
@@ -130,6 +147,40 @@ void decompose_rows(const float *W, int64_t K, int64_t k_n, int64_t r0, int64_t 
                 E[g * kGroup + j] = x - (c - z) * s;
             }
         }
+    }
+    return true;
+}
+
+// D4 for row n over its residual columns cols[0..cnt) (ascending), written
+// at d.col/d.qr[base..base+cnt).
+bool residual_row(const double *E, const int32_t *cols, int64_t cnt, int64_t n, int64_t base,
+                  HostDecomp &d, RowError &err) {
+    double a = 0.0;
+    for (int64_t e = 0; e < cnt; ++e) a = std::max(a, std::fabs(E[cols[e]]));
+    uint16_t srb = f64_to_f16_bits(a / 7.0);
+    if ((srb & 0x7FFF) == 0x7C00) {
+        err.bad = true;
+        err.msg = "a residual scale overflows fp16";
+        return false;
+    }
+    if (srb == 0) srb = 0x3C00;
+    const double sr = f16_bits_to_f64(srb);
+    d.sr[n] = srb;
+    for (int64_t e = 0; e < cnt; ++e) {
+        const int32_t c = cols[e];
+        d.col[base + e] = c;
+        d.qr[base + e] = static_cast<int8_t>(std::min(std::max(std::nearbyint(E[c] / sr), -8.0), 7.0));
+    }
+    return true;
+}
+
+// Row mode: decompose rows [r0, r1) of W into d (already sized).
+void decompose_rows(const float *W, int64_t K, int64_t k_n, int64_t r0, int64_t r1,
+                    HostDecomp &d, RowError &err) {
+    std::vector<double> E(K), absE(K);
+    std::vector<int32_t> idx(K);
+    for (int64_t n = r0; n < r1; ++n) {
+        if (!base_row(W, K, n, d, E.data(), err)) return;
         // residual: the k_n largest |E|, ties to the smaller column
         int64_t base = n * k_n;
         if (k_n > 0) {
@@ -140,37 +191,139 @@ void decompose_rows(const float *W, int64_t K, int64_t k_n, int64_t r0, int64_t 
             };
             if (k_n < K) std::nth_element(idx.begin(), idx.begin() + k_n, idx.end(), before);
             std::sort(idx.begin(), idx.begin() + k_n);
-            double a = 0.0;
-            for (int64_t e = 0; e < k_n; ++e) a = std::max(a, absE[idx[e]]);
-            uint16_t srb = f64_to_f16_bits(a / 7.0);
-            if ((srb & 0x7FFF) == 0x7C00) {
-                err.bad = true;
-                err.msg = "a residual scale overflows fp16";
-                return;
-            }
-            if (srb == 0) srb = 0x3C00;
-            double sr = f16_bits_to_f64(srb);
-            d.sr[n] = srb;
-            for (int64_t e = 0; e < k_n; ++e) {
-                int32_t c = idx[e];
-                double r = std::min(std::max(std::nearbyint(E[c] / sr), -8.0), 7.0);
-                d.col[base + e] = c;
-                d.qr[base + e] = static_cast<int8_t>(r);
-            }
+            if (!residual_row(E.data(), idx.data(), k_n, n, base, d, err)) return;
         } else {
             d.sr[n] = 0x3C00;
         }
     }
 }
 
+// Block mode, pass 1: the base of the rows of row-blocks [b0, b1) and the
+// delta score of each of their 16 x 64 blocks.
+void score_blocks(const float *W, int64_t K, const float *h, int64_t b0, int64_t b1, HostDecomp &d,
+                  std::vector<double> &score, RowError &err) {
+    const int64_t nbc = K / kBlockCols;
+    std::vector<double> E(kBlockRows * K);
+    for (int64_t rb = b0; rb < b1; ++rb) {
+        for (int r = 0; r < kBlockRows; ++r)
+            if (!base_row(W, K, rb * kBlockRows + r, d, E.data() + r * K, err)) return;
+        for (int64_t cb = 0; cb < nbc; ++cb) {
+            double acc = 0.0;  // row by row, column by column
+            for (int r = 0; r < kBlockRows; ++r)
+                for (int c = 0; c < kBlockCols; ++c) {
+                    const int64_t k = cb * kBlockCols + c;
+                    const double e = E[r * K + k];
+                    const double t = e * e;
+                    const double w = h ? static_cast<double>(h[k]) : 1.0;
+                    const double term = t * w;
+                    acc = acc + term;
+                }
+            score[rb * nbc + cb] = acc;
+        }
+    }
+}
+
+// Block mode, pass 2: the residual of the rows of row-blocks [b0, b1) over
+// the columns of their selected blocks (sel[rb * nbc + cb]).
+void block_residual(const float *W, int64_t K, int64_t b0, int64_t b1, const std::vector<uint8_t> &sel,
+                    HostDecomp &d, RowError &err) {
+    const int64_t nbc = K / kBlockCols;
+    std::vector<double> E(K);
+    std::vector<int32_t> cols;
+    for (int64_t rb = b0; rb < b1; ++rb) {
+        cols.clear();
+        for (int64_t cb = 0; cb < nbc; ++cb)
+            if (sel[rb * nbc + cb])
+                for (int c = 0; c < kBlockCols; ++c) cols.push_back(static_cast<int32_t>(cb * kBlockCols + c));
+        for (int r = 0; r < kBlockRows; ++r) {
+            const int64_t n = rb * kBlockRows + r;
+            if (cols.empty()) {
+                d.sr[n] = 0x3C00;
+                continue;
+            }
+            if (!base_row(W, K, n, d, E.data(), err)) return;
+            if (!residual_row(E.data(), cols.data(), static_cast<int64_t>(cols.size()), n, d.row_ptr[n], d,
+                              err))
+                return;
+        }
+    }
+}
+
+template <class F>
+void parallel_rows(int64_t units, F &&body, std::vector<RowError> &errs) {
+    unsigned hw = std::max(1u, std::thread::hardware_concurrency());
+    int64_t nthreads = std::min<int64_t>(std::min<int64_t>(hw, 32), std::max<int64_t>(1, units / 4));
+    errs.assign(nthreads, RowError());
+    std::vector<std::thread> pool;
+    int64_t chunk = (units + nthreads - 1) / nthreads;
+    for (int64_t t = 0; t < nthreads; ++t) {
+        int64_t u0 = t * chunk, u1 = std::min(units, u0 + chunk);
+        if (u0 >= u1) continue;
+        pool.emplace_back([&, t, u0, u1] { body(u0, u1, errs[t]); });
+    }
+    for (auto &th : pool) th.join();
+}
+
+mq_status decompose_blocks_host(const float *W, int64_t N, int64_t K, const mq_pack_opts &opts,
+                                HostDecomp &d) {
+    const int64_t G = K / kGroup, nbr = N / kBlockRows, nbc = K / kBlockCols;
+    const int64_t nsel = residual_blocks_selected(N, K, opts.block_fraction);
+    std::vector<double> score;
+    std::vector<uint8_t> sel;
+    try {
+        d.q.assign(N * K, 0);
+        d.s.assign(N * G, 0);
+        d.z.assign(N * G, 0);
+        d.row_ptr.assign(N + 1, 0);
+        d.sr.assign(N, 0x3C00);
+        score.assign(nbr * nbc, 0.0);
+        sel.assign(nbr * nbc, 0);
+    } catch (const std::bad_alloc &) {
+        return fail(MQ_ERR_OUT_OF_MEMORY, "host allocation for the decomposition failed");
+    }
+    std::vector<RowError> errs;
+    parallel_rows(nbr, [&](int64_t b0, int64_t b1, RowError &e) {
+        score_blocks(W, K, opts.channel_weight, b0, b1, d, score, e);
+    }, errs);
+    for (auto &e : errs)
+        if (e.bad) return fail(MQ_ERR_INVALID_ARG, e.msg);
+    // the nsel largest scores, ties to the smaller block index
+    std::vector<int64_t> order(nbr * nbc);
+    std::iota(order.begin(), order.end(), int64_t(0));
+    auto before = [&](int64_t a, int64_t b) { return score[a] > score[b] || (score[a] == score[b] && a < b); };
+    if (nsel < nbr * nbc) std::nth_element(order.begin(), order.begin() + nsel, order.end(), before);
+    for (int64_t i = 0; i < nsel; ++i) sel[order[i]] = 1;
+    for (int64_t rb = 0; rb < nbr; ++rb) {
+        int64_t cnt = 0;
+        for (int64_t cb = 0; cb < nbc; ++cb) cnt += sel[rb * nbc + cb];
+        for (int r = 0; r < kBlockRows; ++r) {
+            const int64_t n = rb * kBlockRows + r;
+            d.row_ptr[n + 1] = d.row_ptr[n] + cnt * kBlockCols;
+        }
+    }
+    try {
+        d.col.assign(d.row_ptr[N], 0);
+        d.qr.assign(d.row_ptr[N], 0);
+    } catch (const std::bad_alloc &) {
+        return fail(MQ_ERR_OUT_OF_MEMORY, "host allocation for the decomposition failed");
+    }
+    parallel_rows(nbr, [&](int64_t b0, int64_t b1, RowError &e) { block_residual(W, K, b0, b1, sel, d, e); },
+                  errs);
+    for (auto &e : errs)
+        if (e.bad) return fail(MQ_ERR_INVALID_ARG, e.msg);
+    return MQ_OK;
+}
+
 }  // namespace
 
-mq_status decompose_host(const float *W, int64_t N, int64_t K, double rho, HostDecomp &d) {
+mq_status decompose_host(const float *W, int64_t N, int64_t K, const mq_pack_opts &opts, HostDecomp &d) {
     if (std::fegetround() != FE_TONEAREST)
         return fail(MQ_ERR_UNSUPPORTED, "the host FPU rounding mode must be round-to-nearest");
-    const int64_t G = K / kGroup, k_n = residual_count(K, rho);
     d.N = N;
     d.K = K;
+    if (opts.residual_blocks == 1) return decompose_blocks_host(W, N, K, opts, d);
+    const double rho = opts.residual_density;
+    const int64_t G = K / kGroup, k_n = residual_count(K, rho);
     try {
         d.q.assign(N * K, 0);
         d.s.assign(N * G, 0);
@@ -215,7 +368,7 @@ mq_decomp view_of(const HostDecomp &d) {
 
 mq_status validate_decomp(const mq_decomp *d) {
     if (!d) return fail(MQ_ERR_INVALID_ARG, "decomposition is NULL");
-    mq_pack_opts o{kGroup, 0.0};
+    mq_pack_opts o{kGroup, 0.0, 0, 0.0, nullptr};
     if (mq_status st = check_shape(d->N, d->K, &o)) return st;
     if (!d->q || !d->s || !d->z || !d->row_ptr || !d->sr)
         return fail(MQ_ERR_INVALID_ARG, "a decomposition array is NULL");

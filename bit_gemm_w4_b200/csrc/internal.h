@@ -10,6 +10,7 @@
 namespace mq {
 
 constexpr int kGroup = 128;
+constexpr int kBlockRows = 16, kBlockCols = 64;  // residual blocks (block mode)
 
 // Thread-local "last error" text behind mq_last_error().
 void set_error(const std::string &msg);
@@ -46,8 +47,9 @@ struct HostPacked {
 
 mq_status check_shape(int64_t N, int64_t K, const mq_pack_opts *opts);
 int64_t residual_count(int64_t K, double rho);
-mq_status decompose_host(const float *W, int64_t N, int64_t K, double rho,
+mq_status decompose_host(const float *W, int64_t N, int64_t K, const mq_pack_opts &opts,
                          HostDecomp &d);
+int64_t residual_blocks_selected(int64_t N, int64_t K, double fraction);
 mq_status validate_decomp(const mq_decomp *d);
 void pack_host(const mq_decomp &d, HostPacked &p);
 mq_decomp view_of(const HostDecomp &d);

@@ -28,7 +28,9 @@ class MQError(RuntimeError):
 
 
 class _PackOpts(ctypes.Structure):
-    _fields_ = [("group_size", ctypes.c_int32), ("residual_density", ctypes.c_double)]
+    _fields_ = [("group_size", ctypes.c_int32), ("residual_density", ctypes.c_double),
+                ("residual_blocks", ctypes.c_int32), ("block_fraction", ctypes.c_double),
+                ("channel_weight", ctypes.c_void_p)]
 
 
 class _Decomp(ctypes.Structure):
@@ -92,8 +94,16 @@ def _check(status: int, where: str):
         raise MQError(status, where, detail)
 
 
-def _opts(rho: float, group: int = 128) -> _PackOpts:
-    return _PackOpts(group, float(rho))
+def _opts(rho: float, group: int = 128, block_fraction=None, channel_weight=None):
+    """Pack options: row mode (rho) unless block_fraction is given, which
+    selects block mode. Returns (options, kept) where kept holds the arrays
+    the options point at for the duration of the call."""
+    if block_fraction is None:
+        return _PackOpts(group, float(rho), 0, 0.0, None), None
+    h = None
+    if channel_weight is not None:
+        h = np.ascontiguousarray(channel_weight, dtype=np.float32)
+    return _PackOpts(group, 0.0, 1, float(block_fraction), None if h is None else h.ctypes.data), h
 
 
 def _ptr(a: np.ndarray) -> int:
@@ -109,10 +119,10 @@ def _stream(stream) -> int:
     return stream.cuda_stream
 
 
-def residual_nnz(N: int, K: int, rho: float, group: int = 128) -> int:
+def residual_nnz(N: int, K: int, rho: float, group: int = 128, *, block_fraction=None) -> int:
     out = ctypes.c_int64()
-    _check(_lib.mq_residual_nnz(N, K, ctypes.byref(_opts(rho, group)), ctypes.byref(out)),
-           "mq_residual_nnz")
+    o, _ = _opts(rho, group, block_fraction)
+    _check(_lib.mq_residual_nnz(N, K, ctypes.byref(o), ctypes.byref(out)), "mq_residual_nnz")
     return out.value
 
 
@@ -125,14 +135,17 @@ def _alloc_packed(N: int, K: int, nnz: int):
     return arrs, hp
 
 
-def pack_host(W: np.ndarray, rho: float, group: int = 128) -> dict:
-    """Decompose and pack on the host (no CUDA call). Returns the packed arrays."""
+def pack_host(W: np.ndarray, rho: float, group: int = 128, *, block_fraction=None,
+              channel_weight=None) -> dict:
+    """Decompose and pack on the host (no CUDA call). Returns the packed arrays.
+    block_fraction selects block mode (see mq_pack_opts)."""
     W = np.ascontiguousarray(W, dtype=np.float32)
     N, K = W.shape
-    nnz = residual_nnz(N, K, rho, group)
+    nnz = residual_nnz(N, K, rho, group, block_fraction=block_fraction)
     arrs, hp = _alloc_packed(N, K, nnz)
-    _check(_lib.mq_pack_host(_ptr(W), N, K, ctypes.byref(_opts(rho, group)), ctypes.byref(hp)),
-           "mq_pack_host")
+    o, keep = _opts(rho, group, block_fraction, channel_weight)
+    _check(_lib.mq_pack_host(_ptr(W), N, K, ctypes.byref(o), ctypes.byref(hp)), "mq_pack_host")
+    del keep
     return arrs
 
 
@@ -143,12 +156,19 @@ class Weight:
         self._h = handle
 
     @classmethod
-    def pack(cls, W: np.ndarray, rho: float, group: int = 128, stream=None) -> "Weight":
+    def pack(cls, W: np.ndarray, rho: float = 0.0, group: int = 128, stream=None, *,
+             block_fraction=None, channel_weight=None) -> "Weight":
+        """Decompose, pack and upload fp32 W [N, K]. Row mode keeps k_n =
+        floor(rho*K + 0.5) residual entries per row; block_fraction selects
+        block mode (16x64 blocks ranked by the channel-weighted squared error,
+        channel_weight = K diagonal-Hessian weights or None for all ones)."""
         W = np.ascontiguousarray(W, dtype=np.float32)
         N, K = W.shape
         h = ctypes.c_void_p()
-        _check(_lib.mq_pack(_ptr(W), N, K, ctypes.byref(_opts(rho, group)), _stream(stream),
-                            ctypes.byref(h)), "mq_pack")
+        o, keep = _opts(rho, group, block_fraction, channel_weight)
+        _check(_lib.mq_pack(_ptr(W), N, K, ctypes.byref(o), _stream(stream), ctypes.byref(h)),
+               "mq_pack")
+        del keep
         return cls(h.value)
 
     @classmethod

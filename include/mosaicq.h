@@ -66,7 +66,26 @@ typedef enum {
 
 typedef struct {
     int32_t group_size;      /* must be 128, else MQ_ERR_UNSUPPORTED */
-    double residual_density; /* rho in [0, 1]; k_n = floor(rho*K + 0.5) per row */
+    double residual_density; /* rho in [0, 1]; k_n = floor(rho*K + 0.5) per row
+                                (row mode only) */
+    /* Residual allocation ("Methodology" 2, Block-Wise Residual Allocation):
+     * 0 = row mode: each row keeps its k_n largest |W - deq| entries;
+     * 1 = block mode: W is cut into 16-row x 64-column blocks, each scored by
+     *     the Hessian-weighted squared error it would remove,
+     *       delta(b) = sum over (n, k) in b of (E[n][k] * E[n][k]) * h[k]
+     *     (E = W - deq, h = channel_weight, summed in fp64 row by row, column
+     *     by column), and the floor(block_fraction * blocks + 0.5) blocks of
+     *     largest delta (ties to the smaller block index, blocks numbered
+     *     row-block major) carry a residual on every entry. Needs N % 16 == 0.
+     * In both modes a row's residual has one fp16 scale s_r = fp16(max |E| / 7)
+     * over its residual entries and codes clamp(rne(E / s_r), -8, 7). */
+    int32_t residual_blocks;
+    double block_fraction;       /* block mode: in [0, 1] */
+    const float *channel_weight; /* block mode: K finite weights >= 0, the
+                                    diagonal Hessian estimate of the input
+                                    channels (sum over calibration tokens of
+                                    x_k^2); NULL weighs every channel 1.
+                                    Read during the call only. */
 } mq_pack_opts;
 
 /* One decomposition in unpacked host form (caller-owned arrays). */
@@ -106,8 +125,10 @@ typedef struct {
  * current device on `stream`. Returns after the upload completed; W may be
  * freed then. *out = NULL on any error.
  * Errors: INVALID_ARG for NULL pointers, N or K <= 0, K % 128 != 0,
- * K > 65536, rho outside [0, 1], NaN/Inf in W, a scale that overflows fp16;
- * UNSUPPORTED for group_size != 128; OUT_OF_MEMORY; CUDA. */
+ * K > 65536, rho outside [0, 1], NaN/Inf in W, a scale that overflows fp16,
+ * and in block mode N % 16 != 0, block_fraction outside [0, 1] or a negative
+ * or non-finite channel weight; UNSUPPORTED for group_size != 128 or an
+ * unknown residual_blocks; OUT_OF_MEMORY; CUDA. */
 mq_status mq_pack(const float *W_host, int64_t N, int64_t K,
                   const mq_pack_opts *opts, mq_stream stream, mq_weight **out);
 
@@ -168,7 +189,8 @@ void mq_free(mq_weight *w);
 
 /* --- support for tests and benchmarks (not needed for inference) --- */
 
-/* Residual entries a pack with these options produces: N * k_n. */
+/* Residual entries a pack with these options produces: N * k_n in row mode,
+ * (selected blocks) * 1024 in block mode. */
 mq_status mq_residual_nnz(int64_t N, int64_t K, const mq_pack_opts *opts,
                           int64_t *nnz);
 

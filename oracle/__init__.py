@@ -6,7 +6,9 @@ the MosaicQuant pages:
   * decompose.py - inlier-outlier disaggregation W ~= Q(W) + R: a dense 4-bit
     base and a sparse 4-bit residual that patches the worst-quantized entries
     (MosaicQuant, "Methodology", 1. Inlier-Outlier Disaggregation, the
-    equation W_hat ~= Q(W_hat) + R; both parts 4-bit).
+    equation W_hat ~= Q(W_hat) + R; both parts 4-bit), with the residual
+    allocated per row or per block ("Methodology" 2, the Hessian-guided
+    delta score).
   * pack.py      - the device byte layout of that decomposition, and unpack.
   * linear.py    - the product Y = X * W_hat^T, W_hat = deq(Q) + R, as dense
     base plus a CSR loop (the "reduction-add" of ZipperEngine's pipeline) and
@@ -22,7 +24,8 @@ library routines (tests/test_oracle_*.py); none is "parity unpinned".
 
 from .decompose import (Decomposition, decompose, from_arrays, fp16_rne,
                         residual_count, quantize_base, select_residual,
-                        quantize_residual)
+                        quantize_residual, decompose_blocks, block_scores,
+                        select_blocks, blocks_selected)
 from .pack import pack, unpack
 from .linear import dequant_base, w_hat, linear, linear_brute
 from .tolerance import parity_report
@@ -31,4 +34,5 @@ __all__ = [
     "Decomposition", "decompose", "from_arrays", "fp16_rne", "residual_count",
     "quantize_base", "select_residual", "quantize_residual", "pack", "unpack",
     "dequant_base", "w_hat", "linear", "linear_brute", "parity_report",
+    "decompose_blocks", "block_scores", "select_blocks", "blocks_selected",
 ]

@@ -31,6 +31,16 @@ encoding this library implements, step by step:
   D5:        W_hat = deq + scatter(q_r * s_r).
 
 rne is round-half-to-even (numpy.rint).
+
+Block mode ("Methodology" 2, Block-Wise Residual Allocation, with its
+Hessian-guided delta score) replaces D3: W is cut into 16-row x 64-column
+blocks; each block's score is its residual error weighted by the activation
+sensitivity of the input channels, delta(b) = sum (E * E) * h over the block
+(h = a diagonal Hessian estimate, e.g. sum over calibration tokens of x_k^2;
+all ones without one), summed in fp64 row by row and column by column; the
+floor(fraction * blocks + 0.5) largest scores (ties to the smaller block
+index, row-block major) carry a residual on every entry. D4 then quantizes
+each row's residual entries with one scale per row, as above.
 """
 
 from __future__ import annotations
@@ -170,6 +180,80 @@ def decompose(W: np.ndarray, rho: float, group: int = 128,
     qr, sr = quantize_residual(Esel)
     return Decomposition(N, K, group, q, s, z, row_ptr, cols.reshape(-1),
                          qr.reshape(-1), sr)
+
+
+BLOCK_ROWS, BLOCK_COLS = 16, 64
+
+
+def blocks_selected(N: int, K: int, fraction: float) -> int:
+    """floor(fraction * blocks + 0.5) with blocks = (N/16) * (K/64)."""
+    return int(np.floor(float(fraction) * ((N // BLOCK_ROWS) * (K // BLOCK_COLS)) + 0.5))
+
+
+def block_scores(E: np.ndarray, h=None) -> np.ndarray:
+    """The delta score of every 16 x 64 block (block index rb * (K/64) + cb):
+    sum over the block of (E * E) * h[k], accumulated in fp64 in row-major
+    order (cumsum is a sequential sum). h: K channel weights (float32) or
+    None for all ones."""
+    N, K = E.shape
+    nbr, nbc = N // BLOCK_ROWS, K // BLOCK_COLS
+    w = np.ones(K) if h is None else np.asarray(h, np.float32).astype(np.float64)
+    T = (E * E) * w[None, :]
+    T = T.reshape(nbr, BLOCK_ROWS, nbc, BLOCK_COLS).transpose(0, 2, 1, 3)
+    T = T.reshape(nbr * nbc, BLOCK_ROWS * BLOCK_COLS)
+    if T.shape[1] == 0 or T.shape[0] == 0:
+        return np.zeros(nbr * nbc)
+    return np.cumsum(T, axis=1)[:, -1]
+
+
+def select_blocks(score: np.ndarray, n_sel: int) -> np.ndarray:
+    """The n_sel largest scores, ties to the smaller index: bool mask."""
+    order = np.argsort(-score, kind="stable")
+    sel = np.zeros(score.size, dtype=bool)
+    sel[order[:n_sel]] = True
+    return sel
+
+
+def decompose_blocks(W: np.ndarray, block_fraction: float, h=None, group: int = 128,
+                     exact_residual: bool = False) -> Decomposition:
+    """D1, D2, block selection, D4, D5 on fp32 W[N][K] (N % 16 == 0)."""
+    q, s, z, deq = quantize_base(W, group)
+    N, K = q.shape
+    if N % BLOCK_ROWS or K % BLOCK_COLS:
+        raise ValueError("block mode needs N % 16 == 0 and K % 64 == 0")
+    if not 0.0 <= block_fraction <= 1.0:
+        raise ValueError("block_fraction must be in [0, 1]")
+    if h is not None:
+        hv = np.asarray(h, np.float32)
+        if hv.shape != (K,) or not np.all(np.isfinite(hv)) or np.any(hv < 0):
+            raise ValueError("channel weights must be K finite values >= 0")
+    E = W.astype(np.float64) - deq
+    nbr, nbc = N // BLOCK_ROWS, K // BLOCK_COLS
+    sel = select_blocks(block_scores(E, h), blocks_selected(N, K, block_fraction)).reshape(nbr, nbc)
+    counts = np.repeat(sel.sum(axis=1) * BLOCK_COLS, BLOCK_ROWS)
+    row_ptr = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    cols, qrs, exact = [], [], []
+    sr = np.ones(N, np.float16)
+    for rb in range(nbr):
+        cb = np.nonzero(sel[rb])[0]
+        if cb.size == 0:
+            continue
+        c = (cb[:, None] * BLOCK_COLS + np.arange(BLOCK_COLS)[None, :]).reshape(-1)
+        Esel = E[rb * BLOCK_ROWS:(rb + 1) * BLOCK_ROWS][:, c]
+        cols.append(np.tile(c, BLOCK_ROWS))
+        if exact_residual:
+            exact.append(Esel.reshape(-1))
+            continue
+        qr, s_r = quantize_residual(Esel)
+        qrs.append(qr.reshape(-1))
+        sr[rb * BLOCK_ROWS:(rb + 1) * BLOCK_ROWS] = s_r
+    col = np.concatenate(cols).astype(np.int64) if cols else np.zeros(0, np.int64)
+    if exact_residual:
+        ex = np.concatenate(exact) if exact else np.zeros(0)
+        return Decomposition(N, K, group, q, s, z, row_ptr, col, np.zeros(col.size, np.int8),
+                             np.ones(N, np.float16), exact=ex)
+    qr = np.concatenate(qrs).astype(np.int8) if qrs else np.zeros(0, np.int8)
+    return Decomposition(N, K, group, q, s, z, row_ptr, col, qr, sr)
 
 
 def from_arrays(d: dict) -> Decomposition:

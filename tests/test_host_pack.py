@@ -61,3 +61,48 @@ def test_subnormal_scales(mq):
     rng = np.random.default_rng(2)
     W = (rng.standard_normal((8, 128)) * 1e-5).astype(np.float32)
     _same(mq, W, 0.03)
+
+
+def _same_blocks(mq, W, fraction, h=None):
+    got = mq.pack_host(W, 0.0, block_fraction=fraction, channel_weight=h)
+    want = oracle.pack(oracle.decompose_blocks(W, fraction, h))
+    for k in ("qweight", "sz", "row_ptr", "col", "val", "rscale"):
+        a, b = np.asarray(got[k]), np.asarray(want[k])
+        assert a.shape == b.shape, k
+        assert np.array_equal(a.view(np.uint8), np.ascontiguousarray(b).view(np.uint8)), k
+
+
+@pytest.mark.parametrize("fraction", [0.0, 0.05, 0.1, 0.3, 1.0])
+def test_block_mode_matches_oracle(mq, fraction):
+    # "Methodology" 2: 16x64 blocks ranked by the delta score, no weights
+    W = synth.weight(256, 1024, std=0.02, outlier_frac=0.005, seed=31)
+    _same_blocks(mq, W, fraction)
+
+
+def test_block_mode_with_calibration_weights(mq):
+    # delta score weighted by a diagonal Hessian estimate from calibration X
+    W, _, _ = synth.workload_inputs("7b_decode", 0, rows=np.arange(512))
+    Xc = synth.activations(64, 4096, seed=5, channels=4, mult=20.0).double().numpy()
+    h = (Xc * Xc).sum(0).astype(np.float32)
+    _same_blocks(mq, W, 0.1, h)
+
+
+def test_block_mode_clustered_columns(mq):
+    # whole outlier columns: the selection concentrates on their blocks
+    W = synth.weight(128, 2048, std=0.015, outlier_frac=0.01, seed=33, outlier_cols=8)
+    _same_blocks(mq, W, 0.1)
+
+
+def test_block_mode_counts_and_errors(mq):
+    assert mq.residual_nnz(256, 1024, 0.0, block_fraction=0.1) == 26 * 1024  # 256 blocks
+    W = np.zeros((24, 256), np.float32)
+    with pytest.raises(mq.MQError) as e:
+        mq.pack_host(W, 0.0, block_fraction=0.1)                 # N % 16 != 0
+    assert e.value.status == 1
+    W = np.zeros((32, 256), np.float32)
+    with pytest.raises(mq.MQError) as e:
+        mq.pack_host(W, 0.0, block_fraction=0.1, channel_weight=-np.ones(256, np.float32))
+    assert e.value.status == 1
+    with pytest.raises(mq.MQError) as e:
+        mq.pack_host(W, 0.0, block_fraction=2.0)
+    assert e.value.status == 1
