@@ -548,14 +548,20 @@ def run_overhead(reps: int):
         return statistics.median(ts)
 
     rows = []
+    # row mode at each density, then block mode ("Methodology" 2) at each
+    # fraction of 16 x 64 blocks (weights: the squared calibration activations)
+    variants = [("row", r) for r in rhos] + [("block", f) for f in (0.025, 0.05, 0.1)]
     for name, N, K, M in cases:
         W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=1)
         X = synth.activations(M, K, seed=2, channels=8, mult=30.0).to(dev)
+        Xc = synth.activations(128, K, seed=3, channels=8, mult=30.0).double()
+        h = (Xc * Xc).sum(0).float().numpy()
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         ws = torch.empty((M, N), dtype=torch.float32, device=dev)
         base = None
-        for rho in rhos:
-            w = mq.Weight.pack(W, rho)
+        for mode, rho in variants:
+            w = (mq.Weight.pack(W, rho) if mode == "row"
+                 else mq.Weight.pack(W, block_fraction=rho, channel_weight=h))
             w.linear(X, Y)
             w.linear_unfused(X, Y, ws)
             torch.cuda.synchronize()
@@ -563,8 +569,9 @@ def run_overhead(reps: int):
             unfused = timed(lambda: w.linear_unfused(X, Y, ws))
             if w.device_error() != 0:
                 raise RuntimeError("device error word set")
-            base = fused if rho == 0.0 else base
-            rows.append({"shape": name, "N": N, "K": K, "M": M, "rho": rho,
+            base = fused if (mode == "row" and rho == 0.0) else base
+            rows.append({"shape": name, "N": N, "K": K, "M": M, "mode": mode,
+                         "rho" if mode == "row" else "block_fraction": rho,
                          "nnz": w.info()["nnz"], "fused_us": round(fused, 2),
                          "unfused_us": round(unfused, 2),
                          "fused_overhead_vs_rho0": round(fused / base - 1.0, 4),
@@ -573,11 +580,56 @@ def run_overhead(reps: int):
     print(json.dumps({"overhead": rows, "timing": f"CUDA events, L2 flushed, median of {reps}"}))
 
 
+# ------------------------------------------------------------------ distortion
+def run_distortion():
+    """Output distortion left by the decomposition, as a fraction of what the
+    plain 4-bit base leaves, against the share of weights given a residual:
+    block mode with the delta score weighted by calibration activations
+    ("Methodology" 2), block mode unweighted, and row mode with the same
+    residual entry count. Y comes from the library (bf16), the reference is
+    X W^T in fp64; the bf16 rounding floor is reported beside it. Synthetic
+    weights and activations (no model weights exist here)."""
+    import torch
+    from bit_gemm_w4_b200 import mosaicq as mq, synth
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    N, K = 4096, 4096
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=51)
+    Xc = synth.activations(256, K, seed=52, channels=8, mult=30.0)   # calibration
+    Xe = synth.activations(256, K, seed=53, channels=8, mult=30.0)   # evaluation
+    h = (Xc.double() ** 2).sum(0).float().numpy()
+    Xe_d = Xe.to(dev)
+    Yref = Xe_d.double() @ torch.from_numpy(W).to(dev).double().T
+    floor = float(((Yref.to(torch.bfloat16).double() - Yref) ** 2).sum())
+
+    def dist(w):
+        Y = w.linear(Xe_d)
+        torch.cuda.synchronize()
+        v = float(((Y.double() - Yref) ** 2).sum())
+        w.free()
+        return v
+
+    d0 = dist(mq.Weight.pack(W, 0.0))
+    out = []
+    for f in (0.0, 0.025, 0.05, 0.1, 0.2):
+        rec = {"fraction": f}
+        rec["block_delta_weighted"] = round(dist(mq.Weight.pack(W, block_fraction=f, channel_weight=h)) / d0, 4)
+        rec["block_unweighted"] = round(dist(mq.Weight.pack(W, block_fraction=f)) / d0, 4)
+        rec["row_topk_same_count"] = round(dist(mq.Weight.pack(W, f)) / d0, 4)
+        out.append(rec)
+    print(json.dumps({"distortion_left_vs_base": out, "bf16_floor_vs_base": round(floor / d0, 4),
+                      "shape": [N, K], "tokens": 256,
+                      "data": "synthetic: W ~ N(0,0.02) + 0.5% 0.2*t3 outliers; X ~ N(0,1) with 8 "
+                              "channels x30; separate calibration and evaluation draws"}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
                     help="run one small case a few times (the ncu capture command) and exit")
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--distortion", action="store_true",
+                    help="measure the output distortion left at each residual share and exit")
     ap.add_argument("--overhead", action="store_true",
                     help="measure the residual's fused and unfused overhead over density 0 and exit")
     ap.add_argument("--gpus", type=int, default=1)
@@ -593,6 +645,9 @@ def main(argv=None):
         return
     if args.overhead:
         run_overhead(max(args.reps, 5))
+        return
+    if args.distortion:
+        run_distortion()
         return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -240,3 +240,40 @@ def test_sweep_grid(mq, cuda, shape, rho):
         assert w.device_error() == 0
         r = oracle_check(Y[:, rows], X, d)
         assert r["ok"], (M, r)
+
+
+@pytest.mark.parametrize("M", [1, 16, 300])
+def test_block_mode_parity(mq, cuda, M):
+    # "Methodology" 2: the block-allocated residual through both kernels
+    W = synth.weight(512, 4096, std=0.02, outlier_frac=0.005, seed=41)
+    Xc = synth.activations(64, 4096, seed=42, channels=4, mult=20.0).double().numpy()
+    h = (Xc * Xc).sum(0).astype(np.float32)
+    w = mq.Weight.pack(W, block_fraction=0.1, channel_weight=h)
+    d = oracle.decompose_blocks(W, 0.1, h)
+    _bytes_equal(w.export(), oracle.pack(d))
+    X = synth.activations(M, 4096, seed=M, channels=8, mult=30.0)
+    Y = w.linear(X.cuda())
+    torch.cuda.synchronize()
+    assert w.device_error() == 0
+    r = oracle_check(Y, X, d)
+    assert r["ok"], r
+    Yu = w.linear_unfused(X.cuda())
+    torch.cuda.synchronize()
+    r = oracle_check(Yu, X, d)
+    assert r["ok"], r
+
+
+def test_block_mode_long_rows(mq, cuda):
+    # 10 % of the 16 x 64 blocks of a 1024 x 11008 projection carry a residual
+    N, K = 1024, 11008
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=43)
+    w = mq.Weight.pack(W, block_fraction=0.1)
+    d = oracle.decompose_blocks(W, 0.1)
+    _bytes_equal(w.export(), oracle.pack(d))
+    X = synth.activations(64, K, seed=44)
+    for M in (1, 64):
+        Y = w.linear(X[:M].cuda())
+        torch.cuda.synchronize()
+        assert w.device_error() == 0
+        r = oracle_check(Y, X[:M], d)
+        assert r["ok"], (M, r)
