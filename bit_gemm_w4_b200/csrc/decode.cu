@@ -14,10 +14,15 @@
 //   * Packed codes and scale/zero words go straight from HBM into registers
 //     (16-byte streaming loads, batches of BG groups, double-buffered); the
 //     first batch is in flight before anything else happens.
-//   * Meanwhile all threads stage X (the CTA's K range) and the tile's CSR
-//     slice into shared memory with cp.async, then one thread per (row,
-//     4-token group) walks that row's residual entries in batches of four
-//     and leaves s_r * sum q_r * x in shared memory (the sparse branch).
+//   * Meanwhile all threads stage X (the CTA's K range) and, when it is
+//     small enough, the tile's CSR slice into shared memory with cp.async.
+//   * Sparse branch, a warp-cooperative CSR walk: a team of THREADS/BN
+//     consecutive lanes owns one row. Its lanes split the tokens into groups
+//     of four and stride over the row's entries in this CTA's K range (a
+//     binary search on the ascending columns finds that range when K is
+//     split); the partial sums meet in a shuffle reduction and s_r * sum
+//     q_r * x is left in shared memory. Long rows (a block-allocated
+//     residual) are spread over the team instead of one thread.
 //   * Dense branch: each group's nibbles become exact bf16 codes (q - z) in
 //     registers (OR into the mantissa of 128.0, subtract 128 + z), 8
 //     mma.sync m16n8k16 accumulate the exact products in fp32, and s times
@@ -34,6 +39,8 @@
 // Launches use programmatic dependent launch: the weight stream (which no
 // earlier kernel writes) starts at once; griddepcontrol.wait precedes the
 // first read of X and the first write of Y.
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
@@ -53,7 +60,7 @@ struct DecodeParams {
     const uint8_t *val;
     const uint16_t *rscale;
     int M, N, K, G, Gp;
-    int csr_cap;  // residual entries the shared-memory slice can hold
+    int csr_cap;  // residual entries staged in shared memory (0: read from global)
     int with_residual;
 };
 
@@ -63,8 +70,14 @@ struct Cfg {
     static constexpr int BN = 16 * RT;       // rows per CTA
     static constexpr int WARPS = RT * S;
     static constexpr int THREADS = WARPS * 32;
-    static constexpr int TG = (MX + 3) / 4;  // residual token groups of 4
-    static_assert(BN * TG <= THREADS, "one thread per (row, token group)");
+    // sparse branch: a team of TEAM lanes per row, TG token groups of TPG
+    // tokens, E lanes per group striding over the row's entries
+    static constexpr int TEAM = THREADS / BN;
+    static constexpr int TPG = MX < 4 ? MX : 4;
+    static constexpr int TG = MX / TPG;
+    static constexpr int E = TEAM / TG;
+    static_assert(THREADS % BN == 0 && TEAM <= 32 && 32 % TEAM == 0, "row teams inside a warp");
+    static_assert(MX % TPG == 0 && TEAM % TG == 0 && (E & (E - 1)) == 0, "team split");
     static_assert(CS == 1 || CS == 2 || CS == 4 || CS == 8, "cluster size");
 };
 
@@ -129,6 +142,19 @@ __device__ __forceinline__ float ld_dsmem_f32(const void *local, uint32_t rank) 
     return v;
 }
 
+// First index in [lo, hi) whose column is >= key (columns ascend in a row).
+__device__ __forceinline__ int col_lower_bound(const uint16_t *colp, int coff, int lo, int hi,
+                                               int key) {
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (static_cast<int>(colp[mid - coff]) < key)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" :::);
@@ -144,7 +170,7 @@ template <int MX, int RT, int S, int BG, int CS>
 __global__ void __launch_bounds__(Cfg<MX, RT, S, BG, CS>::THREADS)
     decode_kernel(const __grid_constant__ DecodeParams p) {
     using C = Cfg<MX, RT, S, BG, CS>;
-    constexpr int NT = C::NT, BN = C::BN, TG = C::TG;
+    constexpr int NT = C::NT, BN = C::BN;
     extern __shared__ __align__(16) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -187,17 +213,22 @@ __global__ void __launch_bounds__(Cfg<MX, RT, S, BG, CS>::THREADS)
     // ---------------------------------------------- stage X and the CSR slice
     float *red = reinterpret_cast<float *>(smem + L.red);
     float *res = reinterpret_cast<float *>(smem + L.res);
-    const uint16_t *col_s = reinterpret_cast<const uint16_t *>(smem + L.col);
-    const uint8_t *val_s = smem + L.val;
-    int e_b = 0, e_e = 0;
+    const int r_t = threadIdx.x / C::TEAM, tl = threadIdx.x % C::TEAM;
+    const int row_t = n0 + r_t;
+    int e_b = 0, e_e = 0, ra = 0, rb = 0;
     if (p.with_residual) {
         e_b = p.row_ptr[n0];
         e_e = p.row_ptr[min(n0 + BN, N)];
+        if (row_t < N) {
+            ra = p.row_ptr[row_t];
+            rb = p.row_ptr[row_t + 1];
+        }
     }
+    const bool staged = p.csr_cap > 0;
     const int col_base = e_b & ~7, val_base = (e_b >> 1) & ~15;
-    {
-        const int ncol16 = (e_e > e_b) ? ((e_e - col_base) * 2 + 15) / 16 : 0;
-        const int nval16 = (e_e > e_b) ? (((e_e + 1) >> 1) - val_base + 15) / 16 : 0;
+    if (staged && e_e > e_b) {
+        const int ncol16 = ((e_e - col_base) * 2 + 15) / 16;
+        const int nval16 = (((e_e + 1) >> 1) - val_base + 15) / 16;
         for (int i = threadIdx.x; i < ncol16; i += C::THREADS)
             cp_async16(smem + L.col + 16 * i, p.col + col_base + 8 * i);
         for (int i = threadIdx.x; i < nval16; i += C::THREADS)
@@ -205,56 +236,70 @@ __global__ void __launch_bounds__(Cfg<MX, RT, S, BG, CS>::THREADS)
     }
     pdl_wait();  // X may come from the previous kernel; Y may still be read by it
     {
-        const int k_lo = g_lo * 128, kcols = (g_hi - g_lo) * 128;
-        const int per_row = kcols / 8;
-        for (int i = threadIdx.x; i < M * per_row; i += C::THREADS) {
-            const int m = i / per_row, c = i % per_row;
-            cp_async16(smem + L.x + m * L.xrs + 16 * c,
-                       p.X + static_cast<size_t>(m) * K + k_lo + 8 * c);
-        }
+        const int k_lo = g_lo * 128, per_row = (g_hi - g_lo) * 16;  // 16-byte chunks
+        for (int m = 0; m < M; ++m)
+            for (int c = threadIdx.x; c < per_row; c += C::THREADS)
+                cp_async16(smem + L.x + m * L.xrs + 16 * c,
+                           p.X + static_cast<size_t>(m) * K + k_lo + 8 * c);
     }
     cp_async_wait_all();
     __syncthreads();
 
     // ---------------------------------------------- sparse branch
-    if (threadIdx.x < BN * TG) {
-        const int r = threadIdx.x / TG, tg = threadIdx.x % TG;
-        const int row = n0 + r;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+        constexpr int E = C::E, TPG = C::TPG;
+        const uint16_t *colp =
+            staged ? reinterpret_cast<const uint16_t *>(smem + L.col) : p.col;
+        const uint8_t *valp = staged ? smem + L.val : p.val;
+        const int coff = staged ? col_base : 0, voff = staged ? val_base : 0;
+        const int tg = tl / E, el = tl % E;
+        float acc[TPG];
+#pragma unroll
+        for (int j = 0; j < TPG; ++j) acc[j] = 0.f;
         float sr = 0.f;
-        if (p.with_residual && row < N) {
-            sr = half_bits_to_f32(p.rscale[row]);
-            const int a = p.row_ptr[row], b = p.row_ptr[row + 1];
-            const int k_lo = g_lo * 128, k_hi = g_hi * 128;
+        if (rb > ra) {
+            const int k_lo = g_lo * 128;
+            int a = ra, b = rb;
+            if constexpr (CS > 1) {
+                a = col_lower_bound(colp, coff, a, b, k_lo);
+                b = col_lower_bound(colp, coff, a, b, g_hi * 128);
+            }
+            sr = half_bits_to_f32(p.rscale[row_t]);
             const uint16_t *xs = reinterpret_cast<const uint16_t *>(smem + L.x);
-            for (int e = a; e < b; e += 4) {
-                int c[4], q[4];
+            for (int e0 = a + el; e0 < b; e0 += 4 * E) {
+                int c[4];
+                float q[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int idx = e + u;
+                    const int idx = e0 + u * E;
                     const bool ok = idx < b;
-                    const int cc = ok ? static_cast<int>(col_s[idx - col_base]) : -1;
-                    const uint32_t byte = ok ? val_s[(idx >> 1) - val_base] : 0u;
-                    const bool in = ok && cc >= k_lo && cc < k_hi;
-                    c[u] = in ? cc - k_lo : 0;
-                    q[u] = in ? static_cast<int>(((byte >> ((idx & 1) * 4)) & 0xF) ^ 8) - 8 : 0;
+                    c[u] = ok ? static_cast<int>(colp[idx - coff]) - k_lo : 0;
+                    const uint32_t byte = ok ? valp[(idx >> 1) - voff] : 0u;
+                    q[u] = ok ? static_cast<float>(
+                                    static_cast<int>(((byte >> ((idx & 1) * 4)) & 0xF) ^ 8) - 8)
+                              : 0.f;
                 }
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int tok = 4 * tg + j;
+                for (int j = 0; j < TPG; ++j) {
+                    const int tok = tg * TPG + j;
                     if (tok < M) {
                         const uint16_t *xr = xs + tok * (L.xrs / 2);
 #pragma unroll
                         for (int u = 0; u < 4; ++u)
-                            acc[j] = fmaf(static_cast<float>(q[u]), bf16_bits_to_f32(xr[c[u]]),
-                                          acc[j]);
+                            acc[j] = fmaf(q[u], bf16_bits_to_f32(xr[c[u]]), acc[j]);
                     }
                 }
             }
         }
+        // every lane reaches the reduction; E lanes of a token group are adjacent
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (4 * tg + j < MX) res[r * MX + 4 * tg + j] = sr * acc[j];
+        for (int off = E / 2; off > 0; off >>= 1)
+#pragma unroll
+            for (int j = 0; j < TPG; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+        if (el == 0) {
+#pragma unroll
+            for (int j = 0; j < TPG; ++j) res[r_t * MX + tg * TPG + j] = sr * acc[j];
+        }
     }
 
     // ---------------------------------------------- dense branch
@@ -401,12 +446,16 @@ mq_status run(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t st
     p.K = static_cast<int>(d.K);
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
-    p.csr_cap = static_cast<int>(tile_nnz);
     p.with_residual = with_residual ? 1 : 0;
+    // The tile's CSR slice is staged in shared memory while that keeps two
+    // CTAs per SM; a longer slice (a dense or block-allocated residual) is
+    // read from global memory by the walk instead.
+    constexpr int kStagedLimit = 100 * 1024;
+    p.csr_cap = static_cast<int>(std::min<int64_t>(tile_nnz, int64_t(1) << 24));
+    if (Layout(M, p.K, p.G, CS, S, MX, C::BN, p.csr_cap).total > kStagedLimit) p.csr_cap = 0;
     const Layout L(M, p.K, p.G, CS, S, MX, C::BN, p.csr_cap);
     if (L.total > 227 * 1024)
-        return fail(MQ_ERR_UNSUPPORTED,
-                    "decode kernel: X slice plus residual slice exceed shared memory");
+        return fail(MQ_ERR_UNSUPPORTED, "decode kernel: the X slice exceeds shared memory");
     auto kern = decode_kernel<MX, RT, S, BG, CS>;
     static bool configured[64] = {};
     int dev = 0;

@@ -83,14 +83,20 @@ def weight(N: int, K: int, *, std: float, outlier_frac: float, seed: int,
 
 
 def activations(M: int, K: int, *, seed: int, channels: int = 0,
-                mult: float = 1.0):
+                mult: float = 1.0, channel_seed: int | None = None):
     """bf16 X[M][K] ~ N(0, 1) with ``channels`` seeded input channels scaled
-    by ``mult``. Returned as a CPU torch.bfloat16 tensor (RNE from fp32)."""
+    by ``mult``. Returned as a CPU torch.bfloat16 tensor (RNE from fp32).
+
+    The outlier channels are drawn after X from the same generator, unless
+    ``channel_seed`` is given: then they come from a generator of their own,
+    so that several draws of X (calibration and evaluation tokens of one
+    layer) share the same outlier channels."""
     import torch
     rng = np.random.default_rng(seed)
     X = rng.standard_normal((M, K), dtype=np.float32)
     if channels > 0:
-        ch = rng.choice(K, channels, replace=False)
+        crng = rng if channel_seed is None else np.random.default_rng(channel_seed)
+        ch = crng.choice(K, channels, replace=False)
         X[:, ch] *= np.float32(mult)
     return torch.from_numpy(X).to(torch.bfloat16)
 

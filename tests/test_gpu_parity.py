@@ -277,3 +277,27 @@ def test_block_mode_long_rows(mq, cuda):
         assert w.device_error() == 0
         r = oracle_check(Y, X[:M], d)
         assert r["ok"], (M, r)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("mode", ["rows", "blocks"])
+def test_long_residual_rows(mq, cuda, M, mode):
+    # Residual rows far longer than a tile's shared-memory slice: the decode
+    # walk reads them from global memory; M = 16 at K = 8192 also splits K
+    # over a cluster, so each rank walks only its column range.
+    N, K = 128, 8192
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=47)
+    if mode == "rows":
+        w = mq.Weight.pack(W, 0.3)
+        d = oracle.decompose(W, 0.3)
+    else:
+        w = mq.Weight.pack(W, block_fraction=0.6)
+        d = oracle.decompose_blocks(W, 0.6)
+    _bytes_equal(w.export(), oracle.pack(d))
+    X = synth.activations(M, K, seed=48 + M, channels=4, mult=20.0)
+    for path in ("auto", "unfused"):
+        Y = w.linear(X.cuda()) if path == "auto" else w.linear_unfused(X.cuda())
+        torch.cuda.synchronize()
+        assert w.device_error() == 0
+        r = oracle_check(Y, X, d)
+        assert r["ok"], (path, r)
