@@ -134,6 +134,45 @@ void build_stage_lists(const HostPacked &hp, std::vector<int32_t> &ptr, std::vec
         }
 }
 
+// The residual grouped per (128-row block, 256-column stage) for the wide
+// decode kernel (layout in kernels.h, DeviceWeight::wide_ptr): inside a
+// slice, entries are ordered by (16-row warp tile, 128-column group, MMA
+// k-step) so that each warp finds the entries of one k-step contiguous.
+void build_wide_lists(const HostPacked &hp, std::vector<int32_t> &ptr, std::vector<uint16_t> &off,
+                      std::vector<uint16_t> &ent, int64_t &max_len) {
+    const int64_t blocks = (hp.N + 127) / 128, S = (hp.K + 255) / 256, keys = blocks * S;
+    // sub-key inside a slice: warp tile (8) x group (2) x k-step (8); the
+    // k-step of column c in its group is (c % 32) / 4 (the nibble interleave)
+    auto sub = [](int64_t n, int64_t c) {
+        return ((n % 128) / 16) * 16 + ((c % 256) / 128) * 8 + (c % 32) / 4;
+    };
+    std::vector<int32_t> cnt(static_cast<size_t>(keys * 128 + 1), 0);
+    for (int64_t n = 0; n < hp.N; ++n)
+        for (int64_t e = hp.row_ptr[n]; e < hp.row_ptr[n + 1]; ++e) {
+            const int64_t c = hp.col[e];
+            ++cnt[((n / 128) * S + c / 256) * 128 + sub(n, c) + 1];
+        }
+    for (int64_t k = 0; k < keys * 128; ++k) cnt[k + 1] += cnt[k];
+    ptr.assign(static_cast<size_t>(keys + 1), 0);
+    off.assign(static_cast<size_t>(keys * kWideOffStride), 0);
+    max_len = 0;
+    for (int64_t k = 0; k <= keys; ++k) ptr[k] = cnt[k * 128];
+    for (int64_t k = 0; k < keys; ++k) {
+        for (int u = 0; u <= 128; ++u)
+            off[k * kWideOffStride + u] = static_cast<uint16_t>(cnt[k * 128 + u] - ptr[k]);
+        max_len = std::max<int64_t>(max_len, ptr[k + 1] - ptr[k]);
+    }
+    ent.assign(static_cast<size_t>(hp.nnz), 0);
+    std::vector<int32_t> fill(cnt.begin(), cnt.end() - 1);
+    for (int64_t n = 0; n < hp.N; ++n)
+        for (int64_t e = hp.row_ptr[n]; e < hp.row_ptr[n + 1]; ++e) {
+            const int64_t c = hp.col[e];
+            const uint32_t nib = (hp.val[e >> 1] >> ((e & 1) * 4)) & 0xF;
+            ent[fill[((n / 128) * S + c / 256) * 128 + sub(n, c)]++] =
+                static_cast<uint16_t>((c % 256) | ((n % 16) << 8) | (nib << 12));
+        }
+}
+
 mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **out) {
     *out = nullptr;
     int dev = -1;
@@ -170,6 +209,17 @@ mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **o
         st = upload(w, &sptr, hptr.data(), hptr.size(), 0, stream);
         if (!st) st = upload(w, &sent, hent.data(), hent.size(), 0, stream);
     }
+    int32_t *wptr = nullptr;
+    uint16_t *woff = nullptr, *went = nullptr;
+    std::vector<int32_t> hwptr;
+    std::vector<uint16_t> hwoff, hwent;
+    int64_t wide_max = 0;
+    if (!st && hp.nnz > 0) {
+        build_wide_lists(hp, hwptr, hwoff, hwent, wide_max);
+        st = upload(w, &wptr, hwptr.data(), hwptr.size(), 64, stream);
+        if (!st) st = upload(w, &woff, hwoff.data(), hwoff.size(), 0, stream);
+        if (!st) st = upload(w, &went, hwent.data(), hwent.size(), 64, stream);
+    }
     if (!st) st = upload(w, &err, &zero, 1, 0, stream);
     if (!st) {
         e = cudaStreamSynchronize(stream);
@@ -187,6 +237,10 @@ mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **o
     d.rscale = rs;
     d.stage_ptr = sptr;
     d.stage_ent = sent;
+    d.wide_ptr = wptr;
+    d.wide_off = woff;
+    d.wide_ent = went;
+    d.wide_max = wide_max;
     d.err = err;
     w->host_row_ptr = hp.row_ptr;
     for (int64_t n = 0; n < hp.N; ++n)

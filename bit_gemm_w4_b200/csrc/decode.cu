@@ -111,37 +111,6 @@ __device__ __forceinline__ uint32_t ldg_nc(const uint32_t *p) {
     return v;
 }
 
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile(
-        "barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-            : "memory");
-}
-
-__device__ __forceinline__ float ld_dsmem_f32(const void *local, uint32_t rank) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-                 : "=r"(remote)
-                 : "r"(smem_u32(local)), "r"(rank));
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-    return v;
-}
-
 // First index in [lo, hi) whose column is >= key (columns ascend in a row).
 __device__ __forceinline__ int col_lower_bound(const uint16_t *colp, int coff, int lo, int hi,
                                                int key) {
@@ -155,10 +124,6 @@ __device__ __forceinline__ int col_lower_bound(const uint16_t *colp, int coff, i
     return lo;
 }
 
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" :::);
-}
 
 template <int BG>
 struct Batch {
@@ -515,6 +480,10 @@ mq_status run_cs(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t
 
 mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t stream,
                         float *partial) {
+    if (M > 8) {
+        const mq_status st = launch_decode_wide(w, X, M, Y, stream, partial);
+        if (st != MQ_ERR_UNSUPPORTED) return st;
+    }
     if (M == 1) return run_cs<1, 1, 8, 4>(w, X, M, Y, stream, partial);
     if (M <= 8) return run_cs<8, 2, 4, 2>(w, X, M, Y, stream, partial);
     return run_cs<16, 4, 2, 2>(w, X, M, Y, stream, partial);

@@ -1,0 +1,458 @@
+// Wide decode kernel: Y[M][N] = X[M][K] * W_hat^T for 8 < M <= 16, one fused
+// pass.
+//
+// MosaicQuant "Methodology" 3. (ZipperEngine): the dense 4-bit base and the
+// sparse residual are computed in the same pass over the staged activations
+// and meet in one reduction-add.
+//
+// At 16 tokens X is a quarter as large as the packed codes it meets, so
+// staging a CTA's whole slice of X up front (as the narrow decode kernel
+// does) costs about as much shared-memory fill as the weights, and long K
+// must be split over clusters to fit. This kernel streams instead:
+//   * A CTA owns a 128-row block (8 warps x 16 rows) and walks its K range in
+//     stages of 256 columns through a ring of NS shared-memory slots. A slot
+//     holds one stage of X (up to 16 tokens), the block's packed codes and
+//     scale words for the stage, and the block's residual entries whose
+//     columns fall in the stage (grouped per block and stage on the host).
+//   * Every copy is a cp.async issued NS-1 stages ahead, so the HBM stream
+//     never waits for compute. Codes and scale words are copied by the
+//     threads that read them back; X and the residual by all threads, which
+//     then meet at one barrier per stage.
+//   * Dense branch: warp w turns its 16 rows' nibbles into exact bf16 codes
+//     (q - z), accumulates the products with mma.sync m16n8k16 in fp32 and
+//     rescales each 128-column group by s in fp32.
+//   * Sparse branch, on the tensor cores as well: the host orders a warp's
+//     residual entries of a stage by MMA k-step, so for every k-step that
+//     holds entries the warp's lanes scatter them as exact bf16 codes into a
+//     zeroed 512-byte tile laid out in A-fragment order, read their fragment
+//     back, clear it, and issue one more mma.sync on the X fragments the
+//     dense branch already holds. The cost follows the entry count however
+//     the entries cluster (an outlier-inflated group can put a row's whole
+//     residual in one stage), and k-steps without entries cost nothing. The
+//     fp32 sum is multiplied by s_r at the end.
+//   * Reduction-add: dense sums and s_r times the residual sums meet in a
+//     [128][16] fp32 tile; when the block count alone does not fill the GPU,
+//     a cluster of CS CTAs splits K and rank 0 adds the other ranks' tiles
+//     over DSMEM before the single bf16 store.
+// X rows in a slot are 16 bytes longer than 256 columns, and their 16-byte
+// chunks are permuted (chunk c sits at c ^ 2 * ((c >> 3) & 1)), so the
+// fragment loads of a warp touch distinct banks. The k order inside a group
+// follows the same permutation as the narrow kernel (the nibble interleave
+// of the packed codes), applied to X and W alike.
+//
+// Launches use programmatic dependent launch: codes, scales and residual
+// entries (which no earlier kernel writes) are requested before
+// griddepcontrol.wait; X is read and Y written only after it.
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "kernels.h"
+
+namespace mq {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kBN = 16 * kWarps;             // rows per CTA
+constexpr int kKC = 256;                     // columns per stage (two groups)
+constexpr int kMX = 16;                      // token capacity
+constexpr int kXRS = kKC * 2 + 16;           // X row stride in a slot (bytes)
+constexpr int kXBytes = kMX * kXRS;          // 8448
+constexpr int kWBytes = kBN * (kKC / 2);     // [warp][group][16 rows][64 B]
+constexpr int kSZBytes = kBN * 2 * 4;        // [warp][group][16 rows] u32
+constexpr int kOffBytes = kWideOffStride * 2;
+constexpr int kSmemLimit = 112 * 1024;       // two CTAs per SM
+
+struct WideParams {
+    const uint32_t *qweight;  // [N][K/8]
+    const uint32_t *sz;       // [N][Gp]
+    const __nv_bfloat16 *X;   // [M][K]
+    __nv_bfloat16 *Y;         // [M][N]
+    float *Yf;                // fp32 dense-only output (unfused path) or null
+    const int32_t *wptr;
+    const uint16_t *woff;
+    const uint16_t *went;
+    const uint16_t *rscale;
+    int M, N, K, G, Gp;
+    int S;           // stages over all of K
+    int spr;         // stages per cluster rank
+    int ent_bytes;   // residual entry bytes of one slot; 0 = no residual
+    int slot_bytes;  // bytes of one ring slot
+};
+
+// Bytes in front of the ring: the CTA's slice-start table, copied in 16-byte
+// chunks from a 4-entry-aligned start, then one residual fragment tile per
+// warp.
+__host__ __device__ constexpr int wtab_bytes(int spr) { return ((spr + 8) / 4 + 1) * 16; }
+constexpr int kTileBytes = 512;  // 16 rows x 16 k-slots of bf16, A-fragment order
+__host__ __device__ constexpr int ring_offset(int spr) { return wtab_bytes(spr) + kWarps * kTileBytes; }
+
+// Byte offset in a fragment tile of the code at row r (0..15), column c of a
+// 128-column group: thread (g = r % 8, t = c / 32) holds it in register
+// (r / 8) + 2 * ((c % 4) / 2), half c % 2 (the m16n8k16 A layout under the
+// packed codes' k order, where k-step (c % 32) / 4 covers column c).
+__device__ __forceinline__ int tile_pos(int r, int c) {
+    return (((r & 7) * 4 + (c >> 5)) * 4 + (r >> 3) + 2 * ((c & 3) >> 1)) * 4 + (c & 1) * 2;
+}
+
+__device__ __forceinline__ int xchunk(int c) { return c ^ (((c >> 3) & 1) << 1); }
+
+template <int CS, int NS>
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_wide_kernel(const __grid_constant__ WideParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int M = p.M, N = p.N, K = p.K, G = p.G;
+    const int crank = CS > 1 ? static_cast<int>(cluster_rank()) : 0;
+    const int blk = blockIdx.x / CS;
+    const int n0 = blk * kBN;
+    const int j_lo = min(p.S, crank * p.spr), j_hi = min(p.S, j_lo + p.spr);
+    const int nj = j_hi - j_lo;
+    const bool with_res = p.ent_bytes > 0;
+
+    int32_t *wtab = reinterpret_cast<int32_t *>(smem);
+    const int key0 = blk * p.S + j_lo, kbase = key0 & ~3;
+    uint8_t *const rtile = smem + wtab_bytes(p.spr) + warp * kTileBytes;
+    uint8_t *const slots = smem + ring_offset(p.spr);
+    auto slot_of = [&](int i) { return slots + (i % NS) * p.slot_bytes; };
+
+    // sources of this thread's codes (rows g, g+8 of the warp) and scales
+    const size_t wrow = static_cast<size_t>(K) / 8;
+    const int ra = min(n0 + 16 * warp + g, N - 1), rb = min(n0 + 16 * warp + g + 8, N - 1);
+    const uint32_t *w0 = p.qweight + static_cast<size_t>(ra) * wrow + 4 * t;
+    const uint32_t *w1 = p.qweight + static_cast<size_t>(rb) * wrow + 4 * t;
+    const int zrow = lane & 15, zj = lane >> 4;
+    const uint32_t *szp =
+        p.sz + static_cast<size_t>(min(n0 + 16 * warp + zrow, N - 1)) * p.Gp + zj;
+
+    auto issue_weights = [&](int i) {
+        uint8_t *sl = slot_of(i);
+        const int j = j_lo + i;
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const int gi = 2 * j + jj;
+            if (gi < G) {
+                uint8_t *wd = sl + kXBytes + (warp * 2 + jj) * 16 * 64 + 16 * t;
+                cp_async16(wd + g * 64, w0 + gi * 16);
+                cp_async16(wd + (g + 8) * 64, w1 + gi * 16);
+            }
+        }
+        if (2 * j + zj < G)
+            cp_async4(sl + kXBytes + kWBytes + ((warp * 2 + zj) * 16 + zrow) * 4, szp + 2 * j);
+    };
+    auto issue_residual = [&](int i) {
+        uint8_t *sl = slot_of(i);
+        const int key = blk * p.S + j_lo + i;
+        if (threadIdx.x < kOffBytes / 16)
+            cp_async16(sl + kXBytes + kWBytes + kSZBytes + 16 * threadIdx.x,
+                       p.woff + static_cast<size_t>(key) * kWideOffStride + 8 * threadIdx.x);
+        const int eb = wtab[key - kbase], ee = wtab[key - kbase + 1];
+        const int base = eb & ~7, n16 = (ee - base + 7) >> 3;
+        uint8_t *ed = sl + kXBytes + kWBytes + kSZBytes + kOffBytes;
+        for (int c = threadIdx.x; c < n16; c += kThreads) cp_async16(ed + 16 * c, p.went + base + 8 * c);
+    };
+    auto issue_x = [&](int i) {
+        uint8_t *sl = slot_of(i);
+        const int k0 = (j_lo + i) * kKC;
+        const int chunks = min(kKC, K - k0) / 8;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int idx = threadIdx.x + kThreads * u;
+            const int tok = idx >> 5, c = idx & 31;
+            if (tok < M && c < chunks)
+                cp_async16(sl + tok * kXRS + xchunk(c) * 16,
+                           p.X + static_cast<size_t>(tok) * K + k0 + 8 * c);
+        }
+    };
+
+    // ---------------------------------------------- prologue
+    if (with_res) {
+        const int cnt = key0 + nj + 1 - kbase;
+        for (int c = threadIdx.x; 4 * c < cnt; c += kThreads) cp_async16(wtab + 4 * c, p.wptr + kbase + 4 * c);
+        cp_async_commit();
+    }
+    for (int i = 0; i < NS - 1; ++i)
+        if (i < nj) issue_weights(i);
+    pdl_launch_dependents();
+    if (with_res) {
+        cp_async_wait_group<0>();  // the table only: the copies above are not committed yet
+        __syncthreads();
+        for (int i = 0; i < NS - 1; ++i)
+            if (i < nj) issue_residual(i);
+    }
+    pdl_wait();  // X may come from the previous kernel; Y may still be read by it
+    for (int i = 0; i < NS - 1; ++i) {
+        if (i < nj) issue_x(i);
+        cp_async_commit();
+    }
+
+    // ---------------------------------------------- stages
+    float acc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+    float racc[2][4];  // sparse branch, in the accumulator layout of acc
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) racc[nt][i] = 0.f;
+    sts128(rtile + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
+    __syncwarp();
+
+    for (int i = 0; i < nj; ++i) {
+        cp_async_wait_group<NS - 2>();
+        __syncthreads();  // stage i is visible to all; slot (i - 1) % NS is free
+        if (i + NS - 1 < nj) {
+            issue_weights(i + NS - 1);
+            if (with_res) issue_residual(i + NS - 1);
+            issue_x(i + NS - 1);
+        }
+        cp_async_commit();
+
+        const uint8_t *sl = slot_of(i);
+        const int j = j_lo + i;
+        // dense branch
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const int gi = 2 * j + jj;
+            if (gi >= G) break;
+            const uint8_t *wd = sl + kXBytes + (warp * 2 + jj) * 16 * 64 + 16 * t;
+            const uint4 wa = lds128(wd + g * 64), wb = lds128(wd + (g + 8) * 64);
+            const uint32_t *zs =
+                reinterpret_cast<const uint32_t *>(sl + kXBytes + kWBytes) + (warp * 2 + jj) * 16;
+            const uint32_t sz0 = zs[g], sz1 = zs[g + 8];
+            const float s0 = half_bits_to_f32(sz0), s1 = half_bits_to_f32(sz1);
+            const uint32_t z0 = static_cast<uint32_t>(half_bits_to_f32(sz0 >> 16));
+            const uint32_t z1 = static_cast<uint32_t>(half_bits_to_f32(sz1 >> 16));
+            const uint32_t zz0 = (0x4300u | z0) * 0x00010001u;  // bf16x2 (128+z)
+            const uint32_t zz1 = (0x4300u | z1) * 0x00010001u;
+            uint32_t xb[2][16];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int tok = g + 8 * nt;
+                if (tok < M) {
+                    const uint8_t *xr = sl + tok * kXRS;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 v = lds128(xr + xchunk(16 * jj + 4 * t + q) * 16);
+                        xb[nt][4 * q + 0] = v.x;
+                        xb[nt][4 * q + 1] = v.y;
+                        xb[nt][4 * q + 2] = v.z;
+                        xb[nt][4 * q + 3] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) xb[nt][q] = 0u;
+                }
+            }
+            float c[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) c[nt][q] = 0.f;
+            const uint32_t wr0[4] = {wa.x, wa.y, wa.z, wa.w};
+            const uint32_t wr1[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t a_lo = wr0[ks >> 1] >> (8 * (ks & 1));
+                const uint32_t b_lo = wr1[ks >> 1] >> (8 * (ks & 1));
+                uint32_t a[4];
+                a[0] = bf16x2_sub(nib_pair_bias128(a_lo), zz0);
+                a[1] = bf16x2_sub(nib_pair_bias128(b_lo), zz1);
+                a[2] = bf16x2_sub(nib_pair_bias128(a_lo >> 4), zz0);
+                a[3] = bf16x2_sub(nib_pair_bias128(b_lo >> 4), zz1);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    mma_bf16_16816(c[nt], a, xb[nt][2 * ks], xb[nt][2 * ks + 1], c[nt]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                acc[nt][0] = fmaf(s0, c[nt][0], acc[nt][0]);
+                acc[nt][1] = fmaf(s0, c[nt][1], acc[nt][1]);
+                acc[nt][2] = fmaf(s1, c[nt][2], acc[nt][2]);
+                acc[nt][3] = fmaf(s1, c[nt][3], acc[nt][3]);
+            }
+            // sparse branch: the warp's entries of this group, k-step by k-step
+            if (with_res) {
+                const uint16_t *offw =
+                    reinterpret_cast<const uint16_t *>(sl + kXBytes + kWBytes + kSZBytes) +
+                    warp * 16 + jj * 8;
+                const uint16_t *ent = reinterpret_cast<const uint16_t *>(
+                                          sl + kXBytes + kWBytes + kSZBytes + kOffBytes) +
+                                      (wtab[blk * p.S + j - kbase] & 7);
+                int a = lds_u16(offw);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int b = lds_u16(offw + ks + 1);
+                    if (b > a) {  // the same for every lane
+                        for (int e = a + lane; e < b; e += 32) {
+                            const uint32_t v = lds_u16(ent + e);
+                            const int q = static_cast<int>(((v >> 12) & 0xFu) ^ 8u) - 8;
+                            sts_u16(rtile + tile_pos(static_cast<int>((v >> 8) & 0xFu),
+                                                     static_cast<int>(v & 0x7Fu)),
+                                    __float_as_uint(static_cast<float>(q)) >> 16);
+                        }
+                        __syncwarp();
+                        const uint4 f = lds128(rtile + 16 * lane);
+                        sts128(rtile + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
+                        __syncwarp();
+                        const uint32_t fa[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+                            mma_bf16_16816(racc[nt], fa, xb[nt][2 * ks], xb[nt][2 * ks + 1], racc[nt]);
+                    }
+                    a = b;
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------- reduction-add
+    cp_async_wait_all();
+    __syncthreads();  // every slot is idle: the result tile reuses them
+    float *res = reinterpret_cast<float *>(slots);  // [kBN][kMX]
+    float sra = 0.f, srb = 0.f;
+    if (with_res) {
+        const int na = n0 + 16 * warp + g, nb = na + 8;
+        if (na < N) sra = half_bits_to_f32(p.rscale[na]);
+        if (nb < N) srb = half_bits_to_f32(p.rscale[nb]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int row = 16 * warp + g + ((i < 2) ? 0 : 8);
+            const int tok = 8 * nt + 2 * t + (i & 1);
+            res[row * kMX + tok] = fmaf(i < 2 ? sra : srb, racc[nt][i], acc[nt][i]);
+        }
+
+    if constexpr (CS > 1)
+        cluster_sync();
+    else
+        __syncthreads();
+    if (crank == 0) {
+        for (int idx = threadIdx.x; idx < M * kBN; idx += kThreads) {
+            const int m = idx / kBN, r = idx % kBN, n = n0 + r;
+            float y = res[r * kMX + m];
+            if constexpr (CS > 1) {
+#pragma unroll
+                for (int k = 1; k < CS; ++k) y += ld_dsmem_f32(&res[r * kMX + m], k);
+            }
+            if (n < N) {
+                if (p.Yf)
+                    p.Yf[static_cast<size_t>(m) * N + n] = y;
+                else
+                    p.Y[static_cast<size_t>(m) * N + n] = __float2bfloat16_rn(y);
+            }
+        }
+    }
+    // the other ranks keep their shared memory alive until rank 0 has read it
+    if constexpr (CS > 1) cluster_sync();
+}
+
+int sm_count() {
+    static int sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms[dev] = 148;
+    return sms[dev];
+}
+
+template <int CS, int NS>
+mq_status run(const WideParams &p, int smem, int blocks, cudaStream_t stream) {
+    auto kern = decode_wide_kernel<CS, NS>;
+    static bool configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+            return fail(MQ_ERR_CUDA, "cudaFuncSetAttribute failed for the wide decode kernel");
+        configured[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks * CS));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attrs[2];
+    int na = 0;
+    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (CS > 1) {
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = CS;
+        attrs[na].val.clusterDim.y = 1;
+        attrs[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess)
+        return fail(MQ_ERR_CUDA, std::string("wide decode launch: ") + cudaGetErrorString(e));
+    return MQ_OK;
+}
+
+template <int CS>
+mq_status run_ns(const WideParams &p, int ns, int smem, int blocks, cudaStream_t stream) {
+    switch (ns) {
+        case 4: return run<CS, 4>(p, smem, blocks, stream);
+        case 3: return run<CS, 3>(p, smem, blocks, stream);
+        default: return run<CS, 2>(p, smem, blocks, stream);
+    }
+}
+
+}  // namespace
+
+mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
+                             cudaStream_t stream, float *partial) {
+    if (M <= 8 || M > kMX) return MQ_ERR_UNSUPPORTED;
+    const DeviceWeight &d = weight_device(w);
+    const bool with_res = partial == nullptr && d.nnz > 0;
+    WideParams p;
+    p.qweight = d.qweight;
+    p.sz = d.sz;
+    p.X = static_cast<const __nv_bfloat16 *>(X);
+    p.Y = static_cast<__nv_bfloat16 *>(Y);
+    p.Yf = partial;
+    p.wptr = d.wide_ptr;
+    p.woff = d.wide_off;
+    p.went = d.wide_ent;
+    p.rscale = d.rscale;
+    p.M = M;
+    p.N = static_cast<int>(d.N);
+    p.K = static_cast<int>(d.K);
+    p.G = static_cast<int>(d.G);
+    p.Gp = static_cast<int>(d.Gp);
+    p.S = static_cast<int>((d.K + kKC - 1) / kKC);
+    const int blocks = static_cast<int>((d.N + kBN - 1) / kBN);
+    // split K over a cluster only while the blocks alone leave SMs idle
+    int cs = 1;
+    while (cs < 8 && static_cast<int64_t>(blocks) * cs < sm_count() && 2 * cs <= p.S) cs *= 2;
+    p.spr = (p.S + cs - 1) / cs;
+    p.ent_bytes = with_res ? static_cast<int>(((d.wide_max + 15) / 8 + 1) * 16) : 0;
+    if (with_res && (!d.wide_ptr || !d.wide_off || !d.wide_ent)) return MQ_ERR_UNSUPPORTED;
+    const int raw = kXBytes + kWBytes + kSZBytes + (with_res ? kOffBytes + p.ent_bytes : 0);
+    p.slot_bytes = (raw + 127) / 128 * 128;
+    int ns = 4;
+    while (ns >= 2 && ring_offset(p.spr) + ns * p.slot_bytes > kSmemLimit) --ns;
+    if (ns < 2) return MQ_ERR_UNSUPPORTED;  // a residual slice too long for the ring
+    const int smem = ring_offset(p.spr) + ns * p.slot_bytes;
+    switch (cs) {
+        case 1: return run_ns<1>(p, ns, smem, blocks, stream);
+        case 2: return run_ns<2>(p, ns, smem, blocks, stream);
+        case 4: return run_ns<4>(p, ns, smem, blocks, stream);
+        default: return run_ns<8>(p, ns, smem, blocks, stream);
+    }
+}
+
+}  // namespace mq

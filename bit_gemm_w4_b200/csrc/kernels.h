@@ -12,6 +12,10 @@ struct mq_weight;
 
 namespace mq {
 
+// Row-offset table stride of the wide decode kernel's residual slices: 129
+// u16 offsets padded to 272 bytes, so every table starts 16-byte aligned.
+constexpr int kWideOffStride = 136;
+
 // Device buffers of one packed weight (all on one GPU).
 struct DeviceWeight {
     int64_t N, K, G, Gp, nnz;
@@ -28,6 +32,19 @@ struct DeviceWeight {
     // + quadrant] is the first entry of each group (one more entry at the end).
     const int32_t *stage_ptr;   // [ceil(N/128) * K/64 * 4 + 1], NULL when nnz = 0
     const uint32_t *stage_ent;  // [nnz]
+    // The residual again, grouped for the wide decode kernel: per (128-row
+    // block, 256-column stage) a slice of u16 entries column-in-stage |
+    // row-in-warp-tile << 8 | (q_r & 0xF) << 12, ordered by (block, stage,
+    // 16-row warp tile, 128-column group, MMA k-step) where the k-step of
+    // column c of a group is (c % 32) / 4. wide_ptr[block * S + stage] is the
+    // first entry of a slice (S = ceil(K/256), one more entry at the end);
+    // wide_off[(block * S + stage) * kWideOffStride + u], u = 0..128, is where
+    // sub-list u = warp * 16 + group * 8 + k-step starts inside its slice
+    // (u = 128: the slice length). NULL when nnz = 0.
+    const int32_t *wide_ptr;   // [ceil(N/128) * S + 1]
+    const uint16_t *wide_off;  // [ceil(N/128) * S * kWideOffStride]
+    const uint16_t *wide_ent;  // [nnz] (+ padding)
+    int64_t wide_max;          // longest slice, entries
     int *err;                 // device error word
 };
 
@@ -60,6 +77,13 @@ const DeviceWeight &weight_device(const mq_weight *w);
 // (the unfused path's first half); else Y (bf16) gets the fused result.
 mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t stream,
                         float *partial = nullptr);
+
+// Wide decode kernel (decode_wide.cu) for 8 < M <= 16; `partial` as for
+// decode. Returns MQ_ERR_UNSUPPORTED (without setting an error message) when
+// its stage ring cannot hold a residual slice, and the caller falls back to
+// launch_decode.
+mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
+                             cudaStream_t stream, float *partial = nullptr);
 
 // Prefill kernel (prefill.cu): any M >= 1; `partial` as for decode.
 mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
