@@ -262,6 +262,15 @@ mq_status fail(mq_status s, const std::string &msg) {
 
 const DeviceWeight &weight_device(const mq_weight *w) { return w->d; }
 
+int sm_count() {
+    static int sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms[dev] = 148;
+    return sms[dev];
+}
+
 const MapSet *weight_maps(const mq_weight *w, int bn, int gs) {
     std::lock_guard<std::mutex> lock(w->maps_mu);
     for (auto *m : w->maps)

@@ -31,9 +31,10 @@
 //     residual in one stage), and k-steps without entries cost nothing. The
 //     fp32 sum is multiplied by s_r at the end.
 //   * Reduction-add: dense sums and s_r times the residual sums meet in a
-//     [128][16] fp32 tile; when the block count alone does not fill the GPU,
-//     a cluster of CS CTAs splits K and rank 0 adds the other ranks' tiles
-//     over DSMEM before the single bf16 store.
+//     [128][16] fp32 tile and are stored once as bf16.
+//   * The kernel is used when the 128-row blocks alone fill the GPU (one CTA
+//     per block, two per SM); smaller layers keep the narrow kernel, whose
+//     K split serves them better.
 // X rows in a slot are 16 bytes longer than 256 columns, and their 16-byte
 // chunks are permuted (chunk c sits at c ^ 2 * ((c >> 3) & 1)), so the
 // fragment loads of a warp touch distinct banks. The k order inside a group
@@ -77,7 +78,6 @@ struct WideParams {
     const uint16_t *rscale;
     int M, N, K, G, Gp;
     int S;           // stages over all of K
-    int spr;         // stages per cluster rank
     int ent_bytes;   // residual entry bytes of one slot; 0 = no residual
     int slot_bytes;  // bytes of one ring slot
 };
@@ -99,24 +99,22 @@ __device__ __forceinline__ int tile_pos(int r, int c) {
 
 __device__ __forceinline__ int xchunk(int c) { return c ^ (((c >> 3) & 1) << 1); }
 
-template <int CS, int NS>
+template <int NS>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_wide_kernel(const __grid_constant__ WideParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int M = p.M, N = p.N, K = p.K, G = p.G;
-    const int crank = CS > 1 ? static_cast<int>(cluster_rank()) : 0;
-    const int blk = blockIdx.x / CS;
+    const int blk = blockIdx.x;
     const int n0 = blk * kBN;
-    const int j_lo = min(p.S, crank * p.spr), j_hi = min(p.S, j_lo + p.spr);
-    const int nj = j_hi - j_lo;
+    const int j_lo = 0, nj = p.S;
     const bool with_res = p.ent_bytes > 0;
 
     int32_t *wtab = reinterpret_cast<int32_t *>(smem);
     const int key0 = blk * p.S + j_lo, kbase = key0 & ~3;
-    uint8_t *const rtile = smem + wtab_bytes(p.spr) + warp * kTileBytes;
-    uint8_t *const slots = smem + ring_offset(p.spr);
+    uint8_t *const rtile = smem + wtab_bytes(p.S) + warp * kTileBytes;
+    uint8_t *const slots = smem + ring_offset(p.S);
     auto slot_of = [&](int i) { return slots + (i % NS) * p.slot_bytes; };
 
     // sources of this thread's codes (rows g, g+8 of the warp) and scales
@@ -330,42 +328,22 @@ __global__ void __launch_bounds__(kThreads, 2)
             res[row * kMX + tok] = fmaf(i < 2 ? sra : srb, racc[nt][i], acc[nt][i]);
         }
 
-    if constexpr (CS > 1)
-        cluster_sync();
-    else
-        __syncthreads();
-    if (crank == 0) {
-        for (int idx = threadIdx.x; idx < M * kBN; idx += kThreads) {
-            const int m = idx / kBN, r = idx % kBN, n = n0 + r;
-            float y = res[r * kMX + m];
-            if constexpr (CS > 1) {
-#pragma unroll
-                for (int k = 1; k < CS; ++k) y += ld_dsmem_f32(&res[r * kMX + m], k);
-            }
-            if (n < N) {
-                if (p.Yf)
-                    p.Yf[static_cast<size_t>(m) * N + n] = y;
-                else
-                    p.Y[static_cast<size_t>(m) * N + n] = __float2bfloat16_rn(y);
-            }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < M * kBN; idx += kThreads) {
+        const int m = idx / kBN, r = idx % kBN, n = n0 + r;
+        const float y = res[r * kMX + m];
+        if (n < N) {
+            if (p.Yf)
+                p.Yf[static_cast<size_t>(m) * N + n] = y;
+            else
+                p.Y[static_cast<size_t>(m) * N + n] = __float2bfloat16_rn(y);
         }
     }
-    // the other ranks keep their shared memory alive until rank 0 has read it
-    if constexpr (CS > 1) cluster_sync();
 }
 
-int sm_count() {
-    static int sms[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        sms[dev] = 148;
-    return sms[dev];
-}
-
-template <int CS, int NS>
+template <int NS>
 mq_status run(const WideParams &p, int smem, int blocks, cudaStream_t stream) {
-    auto kern = decode_wide_kernel<CS, NS>;
+    auto kern = decode_wide_kernel<NS>;
     static bool configured[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
@@ -378,37 +356,19 @@ mq_status run(const WideParams &p, int smem, int blocks, cudaStream_t stream) {
         configured[dev] = true;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(blocks * CS));
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = stream;
-    cudaLaunchAttribute attrs[2];
-    int na = 0;
-    attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attrs[na].val.programmaticStreamSerializationAllowed = 1;
-    ++na;
-    if (CS > 1) {
-        attrs[na].id = cudaLaunchAttributeClusterDimension;
-        attrs[na].val.clusterDim.x = CS;
-        attrs[na].val.clusterDim.y = 1;
-        attrs[na].val.clusterDim.z = 1;
-        ++na;
-    }
-    cfg.attrs = attrs;
-    cfg.numAttrs = na;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
     if (e != cudaSuccess)
         return fail(MQ_ERR_CUDA, std::string("wide decode launch: ") + cudaGetErrorString(e));
     return MQ_OK;
-}
-
-template <int CS>
-mq_status run_ns(const WideParams &p, int ns, int smem, int blocks, cudaStream_t stream) {
-    switch (ns) {
-        case 4: return run<CS, 4>(p, smem, blocks, stream);
-        case 3: return run<CS, 3>(p, smem, blocks, stream);
-        default: return run<CS, 2>(p, smem, blocks, stream);
-    }
 }
 
 }  // namespace
@@ -434,24 +394,20 @@ mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
     p.S = static_cast<int>((d.K + kKC - 1) / kKC);
-    const int blocks = static_cast<int>((d.N + kBN - 1) / kBN);
-    // split K over a cluster only while the blocks alone leave SMs idle
-    int cs = 1;
-    while (cs < 8 && static_cast<int64_t>(blocks) * cs < sm_count() && 2 * cs <= p.S) cs *= 2;
-    p.spr = (p.S + cs - 1) / cs;
+    const int64_t blocks = (d.N + kBN - 1) / kBN;
+    if (blocks < sm_count()) return MQ_ERR_UNSUPPORTED;  // the narrow kernel serves small layers
     p.ent_bytes = with_res ? static_cast<int>(((d.wide_max + 15) / 8 + 1) * 16) : 0;
     if (with_res && (!d.wide_ptr || !d.wide_off || !d.wide_ent)) return MQ_ERR_UNSUPPORTED;
     const int raw = kXBytes + kWBytes + kSZBytes + (with_res ? kOffBytes + p.ent_bytes : 0);
     p.slot_bytes = (raw + 127) / 128 * 128;
     int ns = 4;
-    while (ns >= 2 && ring_offset(p.spr) + ns * p.slot_bytes > kSmemLimit) --ns;
+    while (ns >= 2 && ring_offset(p.S) + ns * p.slot_bytes > kSmemLimit) --ns;
     if (ns < 2) return MQ_ERR_UNSUPPORTED;  // a residual slice too long for the ring
-    const int smem = ring_offset(p.spr) + ns * p.slot_bytes;
-    switch (cs) {
-        case 1: return run_ns<1>(p, ns, smem, blocks, stream);
-        case 2: return run_ns<2>(p, ns, smem, blocks, stream);
-        case 4: return run_ns<4>(p, ns, smem, blocks, stream);
-        default: return run_ns<8>(p, ns, smem, blocks, stream);
+    const int smem = ring_offset(p.S) + ns * p.slot_bytes;
+    switch (ns) {
+        case 4: return run<4>(p, smem, static_cast<int>(blocks), stream);
+        case 3: return run<3>(p, smem, static_cast<int>(blocks), stream);
+        default: return run<2>(p, smem, static_cast<int>(blocks), stream);
     }
 }
 

@@ -72,6 +72,9 @@ const PrefillMaps *prefill_maps(const mq_weight *w);
 bool encode_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K, int chunks);
 const DeviceWeight &weight_device(const mq_weight *w);
 
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count();
+
 // Decode kernels (decode.cu): M in [1, 16]. With `partial` set the residual
 // is skipped and the dense base alone is written as fp32 to `partial`
 // (the unfused path's first half); else Y (bf16) gets the fused result.

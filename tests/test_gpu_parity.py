@@ -305,9 +305,10 @@ def test_long_residual_rows(mq, cuda, M, mode):
 
 @pytest.mark.parametrize("M", [9, 13, 16])
 def test_wide_decode_ragged(mq, cuda, M):
-    # 9..16 tokens: ragged 128-row blocks (N = 200) and a last 256-column
-    # stage holding one group (K = 384), fused and unfused
-    W = synth.weight(200, 384, std=0.02, outlier_frac=0.01, seed=53)
+    # 9..16 tokens on a layer tall enough for the wide decode kernel (149
+    # 128-row blocks, the last one ragged) with a last 256-column stage that
+    # holds one group (K = 384), fused and unfused
+    W = synth.weight(19000, 384, std=0.02, outlier_frac=0.01, seed=53)
     X = synth.activations(M, 384, seed=54 + M, channels=2, mult=20.0)
     w, Y = _run(mq, W, X, 0.05)
     d = oracle.decompose(W, 0.05)
