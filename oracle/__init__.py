@@ -14,6 +14,9 @@ the MosaicQuant pages:
     base plus a CSR loop (the "reduction-add" of ZipperEngine's pipeline) and
     as a brute-force triple loop.
   * tolerance.py - the parity metrics used to accept a bf16 GPU output.
+  * w4a4.py      - the W4A4 variant: per-token int4 activation quantization
+    (the pipeline's quantization stage in "Methodology" 3.) and the product
+    from exact integer sums ("Experimental Results" evaluate W4A4).
 
 This package is test infrastructure. Only tests/, __graft_entry__.smoke() and
 bench.py's CPU-baseline / reference arm may import it. The product path
