@@ -626,6 +626,79 @@ def run_distortion():
                               "the outlier channels"}))
 
 
+# ------------------------------------------------------------------ W4A4
+def run_w4a4():
+    """The W4A4 variant against W4A16 on the same packed weights: the three
+    7B decode shapes at M = 1 and the 70B MLP at M = 16. Each path is timed as
+    a CUDA graph of 48 back-to-back calls, weights rotated through copies
+    larger than L2 (the W4A4 call is two launches: quantization, then the
+    fused product). Bytes are the algorithmic bytes of the W4A16 call (packed
+    weight, CSR, bf16 X and Y once). Prints one JSON line."""
+    import torch
+    from bit_gemm_w4_b200 import mosaicq as mq, synth
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    pk, _ = peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    rows = []
+    for name in ("7b_decode", "70b_mlp"):
+        cfg = synth.WORKLOADS[name]
+        for i, (N, K) in enumerate(cfg["shapes"]):
+            per = alg_bytes(cfg["M"], N, K, 0)
+            copies = max(1, int(np.ceil(2.0 * l2 / per)) + 1) if per < 2 * l2 else 1
+            ws = []
+            for c in range(copies):
+                W = synth.weight(N, K, std=cfg["w_std"], outlier_frac=cfg["w_outlier_frac"],
+                                 outlier_cols=cfg["w_outlier_cols"], seed=1000 * (i + 1) + 17 * c)
+                ws.append(mq.Weight.pack(W, cfg["rho"]))
+                del W
+            M = cfg["M"]
+            X = synth.activations(M, K, seed=7 + i, channels=cfg["x_channels"],
+                                  mult=cfg["x_mult"]).to(dev)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            wsp = torch.empty(int(mq._lib.mq_w4a4_workspace_bytes(ws[0]._h, M)), dtype=torch.uint8,
+                              device=dev)
+            nnz = ws[0].info()["nnz"]
+            out = {"shape": f"{N}x{K}", "M": M, "nnz": nnz}
+            for path in ("w4a16", "w4a4"):
+                def call(k):
+                    w = ws[k % copies]
+                    if path == "w4a16":
+                        w.linear_raw(X.data_ptr(), M, Y.data_ptr(), stream=stream)
+                    else:
+                        w.linear_w4a4(X, Y, wsp, stream=stream)
+                with torch.cuda.stream(stream):
+                    for k in range(copies):
+                        call(k)
+                torch.cuda.synchronize()
+                g = torch.cuda.CUDAGraph()
+                n = 48
+                with torch.cuda.graph(g, stream=stream):
+                    for k in range(n):
+                        call(k)
+                with torch.cuda.stream(stream):
+                    g.replay()
+                    torch.cuda.synchronize()
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    for _ in range(5):
+                        g.replay()
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                us = e0.elapsed_time(e1) * 1e3 / (5 * n)
+                by = alg_bytes(M, N, K, nnz)
+                out[path] = {"us": round(us, 3), "TB_s": round(by / us / 1e6, 3),
+                             "frac": round(by / us / 1e3 / pk["hbm_gbs"], 4)}
+                del g
+            rows.append(out)
+            del ws
+            torch.cuda.empty_cache()
+    print(json.dumps({"w4a4_vs_w4a16": rows, "timing": "CUDA graph of 48 calls, mean over 5 replays",
+                      "peak_hbm_gbs": pk["hbm_gbs"]}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
@@ -633,6 +706,8 @@ def main(argv=None):
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--distortion", action="store_true",
                     help="measure the output distortion left at each residual share and exit")
+    ap.add_argument("--w4a4", action="store_true",
+                    help="time the W4A4 variant against W4A16 on the same weights and exit")
     ap.add_argument("--overhead", action="store_true",
                     help="measure the residual's fused and unfused overhead over density 0 and exit")
     ap.add_argument("--gpus", type=int, default=1)
@@ -651,6 +726,9 @@ def main(argv=None):
         return
     if args.distortion:
         run_distortion()
+        return
+    if args.w4a4:
+        run_w4a4()
         return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -524,4 +524,46 @@ mq_status mq_linear(const mq_weight *w, const void *X, int64_t M, void *Y, mq_st
     return mq_linear_path(w, X, M, Y, stream, MQ_PATH_AUTO);
 }
 
+mq_status mq_quantize_activations(const void *X, int64_t M, int64_t K, void *codes, float *scales,
+                                  mq_stream stream) {
+    if (M < 0) return fail(MQ_ERR_INVALID_ARG, "M must be >= 0");
+    if (K <= 0 || K % 8 || K > (int64_t(1) << 30))
+        return fail(MQ_ERR_INVALID_ARG, "K must be a positive multiple of 8");
+    if (M == 0) return MQ_OK;
+    if (M > (int64_t(1) << 31) - 1) return fail(MQ_ERR_INVALID_ARG, "M too large");
+    if (!X || !codes || !scales) return fail(MQ_ERR_INVALID_ARG, "X, codes or scales is NULL");
+    if (!aligned16(X) || !aligned16(codes) || !aligned16(scales))
+        return fail(MQ_ERR_INVALID_ARG, "X, codes and scales must be 16-byte aligned");
+    return launch_quantize(X, M, K, codes, scales, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int64_t mq_w4a4_workspace_bytes(const mq_weight *w, int64_t M) {
+    if (!w || M <= 0) return 0;
+    return (M * w->d.K + 15) / 16 * 16 + (M * 4 + 15) / 16 * 16;
+}
+
+mq_status mq_linear_w4a4(const mq_weight *w, const void *X, int64_t M, void *Y, void *workspace,
+                         size_t workspace_bytes, mq_stream stream) {
+    if (!w) return fail(MQ_ERR_INVALID_ARG, "weight handle is NULL");
+    if (M < 0) return fail(MQ_ERR_INVALID_ARG, "M must be >= 0");
+    if (M == 0) return MQ_OK;
+    if (M > 16) return fail(MQ_ERR_UNSUPPORTED, "W4A4 serves M <= 16 (the decode regime)");
+    if (!X || !Y || !workspace) return fail(MQ_ERR_INVALID_ARG, "X, Y or workspace is NULL");
+    if (!aligned16(X) || !aligned16(Y) || !aligned16(workspace))
+        return fail(MQ_ERR_INVALID_ARG, "X, Y and workspace must be 16-byte aligned");
+    if (workspace_bytes < static_cast<size_t>(mq_w4a4_workspace_bytes(w, M)))
+        return fail(MQ_ERR_INVALID_ARG, "workspace smaller than mq_w4a4_workspace_bytes");
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
+    if (dev != w->device)
+        return fail(MQ_ERR_INVALID_ARG, "the current device is not the device that packed the weight");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int8_t *codes = static_cast<int8_t *>(workspace);
+    float *scales = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                              (M * w->d.K + 15) / 16 * 16);
+    mq_status st = launch_quantize(X, M, w->d.K, codes, scales, s);
+    if (st) return st;
+    return launch_decode_a4(w, codes, scales, static_cast<int>(M), Y, s);
+}
+
 }  // extern "C"

@@ -134,6 +134,22 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// ---------------------------------------------------------------- streaming loads
+// 16 bytes from HBM that no kernel reuses: read-only path, no L1 allocation.
+__device__ __forceinline__ uint4 ldg_stream(const uint32_t *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ldg_nc(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 // ---------------------------------------------------------------- cp.async, clusters, PDL
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
@@ -187,6 +203,21 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" :::);
 }
+
+// ---------------------------------------------------------------- CSR
+// First index in [lo, hi) whose column is >= key (columns ascend in a row).
+__device__ __forceinline__ int col_lower_bound(const uint16_t *colp, int coff, int lo, int hi,
+                                               int key) {
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (static_cast<int>(colp[mid - coff]) < key)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
 
 // ---------------------------------------------------------------- math
 // bf16x2 (128 + q_lo, 128 + q_hi) for the nibble pair at bits [0,4) and

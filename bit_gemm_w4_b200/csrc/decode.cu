@@ -97,34 +97,6 @@ struct Layout {
     }
 };
 
-__device__ __forceinline__ uint4 ldg_stream(const uint32_t *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ uint32_t ldg_nc(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
-}
-
-// First index in [lo, hi) whose column is >= key (columns ascend in a row).
-__device__ __forceinline__ int col_lower_bound(const uint16_t *colp, int coff, int lo, int hi,
-                                               int key) {
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (static_cast<int>(colp[mid - coff]) < key)
-            lo = mid + 1;
-        else
-            hi = mid;
-    }
-    return lo;
-}
-
-
 template <int BG>
 struct Batch {
     uint4 w[BG][2];

@@ -92,6 +92,14 @@ mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
 mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
                          cudaStream_t stream, float *partial = nullptr);
 
+// W4A4 (w4a4.cu): per-token int4 quantization of bf16 X into int8 codes
+// [M][K] and fp32 scales [M]; then the fused W4A4 product for M <= 16 from
+// those codes (Y bf16 [M][N]).
+mq_status launch_quantize(const void *X, int64_t M, int64_t K, void *codes, float *scales,
+                          cudaStream_t stream);
+mq_status launch_decode_a4(const mq_weight *w, const int8_t *codes, const float *xscale, int M,
+                           void *Y, cudaStream_t stream);
+
 // Separate residual kernel (residual.cu): Y = bf16(partial + X * R^T).
 mq_status launch_residual_merge(const mq_weight *w, const void *X, int64_t M,
                                 const float *partial, void *Y, cudaStream_t stream);

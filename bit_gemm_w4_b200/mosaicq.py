@@ -64,6 +64,9 @@ def _load():
         "mq_linear_path": ([vp, vp, i64, vp, vp, ctypes.c_int], st),
         "mq_linear_unfused": ([vp, vp, i64, vp, vp, ctypes.c_size_t, vp], st),
         "mq_linear_unfused_noalloc": ([vp, vp, i64, vp, vp], st),
+        "mq_quantize_activations": ([vp, i64, i64, vp, vp, vp], st),
+        "mq_w4a4_workspace_bytes": ([vp, i64], i64),
+        "mq_linear_w4a4": ([vp, vp, i64, vp, vp, ctypes.c_size_t, vp], st),
         "mq_free": ([vp], None),
         "mq_residual_nnz": ([i64, i64, ctypes.POINTER(_PackOpts), ctypes.POINTER(i64)], st),
         "mq_pack_host": ([vp, i64, i64, ctypes.POINTER(_PackOpts), ctypes.POINTER(_HostPacked)], st),
@@ -149,6 +152,19 @@ def pack_host(W: np.ndarray, rho: float, group: int = 128, *, block_fraction=Non
     return arrs
 
 
+def quantize_activations(X, *, stream=None):
+    """Per-token int4 codes (int8 [M, K]) and fp32 scales [M] of bf16 X on
+    its device (the W4A4 quantization stage)."""
+    import torch
+    X = X.contiguous()
+    M, K = X.shape
+    codes = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    scales = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _check(_lib.mq_quantize_activations(X.data_ptr(), M, K, codes.data_ptr(), scales.data_ptr(),
+                                        _stream(stream)), "mq_quantize_activations")
+    return codes, scales
+
+
 class Weight:
     """A packed weight on the current CUDA device (owns its device buffers)."""
 
@@ -230,6 +246,24 @@ class Weight:
                                       workspace.data_ptr(),
                                       workspace.numel() * workspace.element_size(),
                                       _stream(stream)), "mq_linear_unfused")
+        return Y
+
+    def linear_w4a4(self, X, Y=None, workspace=None, *, stream=None):
+        """The W4A4 variant for M <= 16: per-token int4 activation codes in a
+        caller-owned workspace (mq_w4a4_workspace_bytes), then the fused
+        int4 x int4 pass."""
+        import torch
+        info = self.info()
+        X = X.contiguous()
+        M = X.shape[0]
+        if Y is None:
+            Y = torch.empty((M, info["N"]), dtype=torch.bfloat16, device=X.device)
+        if workspace is None:
+            nbytes = max(16, int(_lib.mq_w4a4_workspace_bytes(self._h, M)))
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=X.device)
+        _check(_lib.mq_linear_w4a4(self._h, X.data_ptr(), M, Y.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(),
+                                   _stream(stream)), "mq_linear_w4a4")
         return Y
 
     def linear_unfused_noalloc(self, X, Y=None, *, stream=None):

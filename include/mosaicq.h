@@ -183,6 +183,43 @@ mq_status mq_linear_unfused(const mq_weight *w, const void *X_dev, int64_t M,
 mq_status mq_linear_unfused_noalloc(const mq_weight *w, const void *X_dev,
                                     int64_t M, void *Y_dev, mq_stream stream);
 
+/* --- W4A4: activations quantized to 4 bits as well ---
+ * MosaicQuant "Methodology" 3. (ZipperEngine) starts its pipeline with a
+ * quantization stage, and "Experimental Results" evaluate the method as
+ * W4A4. The pages fix no activation format; this library reads it as
+ * per-token symmetric int4:
+ *   s_x[m] = fp32(max_k |x[m][k]| / 7), one IEEE fp32 division (1 when the
+ *            token is all zeros);
+ *   c[m][k] = clamp(rne(fp32(x[m][k] / s_x[m])), -8, 7), again one IEEE
+ *            fp32 division and round-half-to-even;
+ *   Y[m][n] = s_x[m] * (sum_g s[n][g] * sum_{k in g} (q - z) * c[m][k]
+ *                       + s_r[n] * sum_{residual entries} q_r * c[m][col]),
+ * the integer sums exact (int32), the scaling in fp32, Y stored as bf16. */
+
+/* The quantization stage alone: per-token scales and codes of bf16 X.
+ * X_dev: bf16 [M][K] row-major, 16-byte aligned, K a positive multiple of 8.
+ * codes_dev: int8 [M][K] row-major, scales_dev: float [M]; both caller-owned
+ * device memory, 16-byte aligned, written asynchronously on `stream`.
+ * M = 0 launches nothing. Errors: INVALID_ARG for NULL or misaligned
+ * pointers with M > 0, M < 0, or K not a positive multiple of 8; CUDA. */
+mq_status mq_quantize_activations(const void *X_dev, int64_t M, int64_t K, void *codes_dev,
+                                  float *scales_dev, mq_stream stream);
+
+/* Device bytes of the workspace mq_linear_w4a4 needs for M tokens of this
+ * weight (the codes and scales of X). 0 for a NULL handle or M <= 0. */
+int64_t mq_w4a4_workspace_bytes(const mq_weight *w, int64_t M);
+
+/* Y[M][N] for the W4A4 reading above: quantizes X into `workspace`, then
+ * one fused pass computes the dense int4 x int4 base (int8 tensor-core MMAs,
+ * exact int32 group sums), the int4 x int4 residual and the scaling.
+ * X, Y as for mq_linear; workspace: caller-owned device memory of at least
+ * mq_w4a4_workspace_bytes(w, M) bytes, 16-byte aligned, not shared with a
+ * concurrent call. Asynchronous, no allocation. M in [0, 16] (the decode
+ * regime): UNSUPPORTED for M > 16. Errors as mq_linear, plus INVALID_ARG for
+ * a NULL, misaligned or too small workspace. */
+mq_status mq_linear_w4a4(const mq_weight *w, const void *X_dev, int64_t M, void *Y_dev,
+                         void *workspace, size_t workspace_bytes, mq_stream stream);
+
 /* Release every buffer of the handle. NULL-safe. Waits for no stream: the
  * caller makes sure no call using the handle is still in flight. */
 void mq_free(mq_weight *w);
