@@ -165,9 +165,18 @@ class DecodeSet:
         self.flops_per_launch = [alg_flops(self.M, N, K, nz)
                                  for (N, K), nz in zip(self.shapes, self.nnz)]
 
-    def launch(self, copy: int, i: int, stream):
+    def launch(self, copy: int, i: int, stream, prefetch: bool = False):
+        """One layer of the step. With prefetch, mq_linear_prefetch brings the
+        next layer's packed weight (the next shape, or the first shape of the
+        next step's copy) into L2 while this one runs."""
         w = self.weights[copy][i]
-        w.linear_raw(self.X[i].data_ptr(), self.M, self.Y[i].data_ptr(), stream=stream)
+        nxt = None
+        if prefetch:
+            nsh = len(self.shapes)
+            nxt = (self.weights[copy][i + 1] if i + 1 < nsh
+                   else self.weights[(copy + 1) % len(self.weights)][0])
+        w.linear_raw(self.X[i].data_ptr(), self.M, self.Y[i].data_ptr(), stream=stream,
+                     next_weight=nxt)
 
 
 def time_graph_steps(torch, ds: DecodeSet, steps: int, warmup: int, stream, chunk: int,
@@ -242,19 +251,31 @@ def time_per_shape(torch, ds: DecodeSet, stream, n: int = 48):
 
 
 def time_e2e(torch, ds: DecodeSet, steps: int, stream, dist_ctx):
-    """The public API with host buffers: per step H2D of X from pinned memory,
-    the fused calls, D2H of Y into pinned memory."""
+    """The public API with host buffers: per step one host-to-device copy of
+    the step's inputs (the three layers' X, packed in one pinned buffer), the
+    fused calls, and one device-to-host copy of the three outputs into pinned
+    memory."""
     copies = len(ds.weights)
-    hx = [x.cpu().pin_memory() for x in ds.X]
-    hy = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for y in ds.Y]
-    h2d = sum(x.numel() * 2 for x in hx)
-    d2h = sum(y.numel() * 2 for y in hy)
+    # each layer's slice starts 16-byte aligned (8 bf16 elements)
+    xs = [(x.numel() + 7) // 8 * 8 for x in ds.X]
+    ys = [(y.numel() + 7) // 8 * 8 for y in ds.Y]
+    xo = np.concatenate([[0], np.cumsum(xs)]).astype(int)
+    yo = np.concatenate([[0], np.cumsum(ys)]).astype(int)
+    hx = torch.zeros(int(xo[-1]), dtype=torch.bfloat16).pin_memory()
+    for i, x in enumerate(ds.X):
+        hx[xo[i]:xo[i] + x.numel()] = x.reshape(-1).cpu()
+    hy = torch.empty(int(yo[-1]), dtype=torch.bfloat16, pin_memory=True)
+    dx = torch.empty(int(xo[-1]), dtype=torch.bfloat16, device=ds.X[0].device)
+    dy = torch.empty(int(yo[-1]), dtype=torch.bfloat16, device=ds.Y[0].device)
+    h2d, d2h = hx.numel() * 2, hy.numel() * 2
+    nsh = len(ds.shapes)
 
     def step(s):
-        for i in range(len(ds.shapes)):
-            ds.X[i].copy_(hx[i], non_blocking=True)
-            ds.launch(s % copies, i, stream)
-            hy[i].copy_(ds.Y[i], non_blocking=True)
+        dx.copy_(hx, non_blocking=True)
+        for i in range(nsh):
+            ds.weights[s % copies][i].linear_raw(dx[xo[i]:].data_ptr(), ds.M,
+                                                 dy[yo[i]:].data_ptr(), stream=stream)
+        hy.copy_(dy, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for s in range(3):

@@ -485,7 +485,14 @@ mq_status mq_linear_path(const mq_weight *w, const void *X, int64_t M, void *Y, 
     if (dev != w->device)
         return fail(MQ_ERR_INVALID_ARG, "the current device is not the device that packed the weight");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (path == MQ_PATH_AUTO) path = (M <= 16) ? MQ_PATH_DECODE : MQ_PATH_PREFILL;
+    if (path == MQ_PATH_AUTO) {
+        if (M <= 16) {
+            // the decode kernels, unless X's slice cannot fit them (very long K)
+            const mq_status st = launch_decode(w, X, static_cast<int>(M), Y, s);
+            if (st != MQ_ERR_UNSUPPORTED) return st;
+        }
+        return launch_prefill(w, X, M, Y, s);
+    }
     switch (path) {
         case MQ_PATH_DECODE:
             if (M > 16) return fail(MQ_ERR_UNSUPPORTED, "the decode kernel serves M <= 16");
@@ -522,6 +529,26 @@ mq_status mq_linear_unfused(const mq_weight *w, const void *X, int64_t M, void *
 
 mq_status mq_linear(const mq_weight *w, const void *X, int64_t M, void *Y, mq_stream stream) {
     return mq_linear_path(w, X, M, Y, stream, MQ_PATH_AUTO);
+}
+
+mq_status mq_linear_prefetch(const mq_weight *w, const void *X, int64_t M, void *Y,
+                             const mq_weight *next, mq_stream stream) {
+    if (!next || M > 16 || M <= 0) return mq_linear_path(w, X, M, Y, stream, MQ_PATH_AUTO);
+    if (!w) return fail(MQ_ERR_INVALID_ARG, "weight handle is NULL");
+    if (!X || !Y) return fail(MQ_ERR_INVALID_ARG, "X or Y is NULL");
+    if (!aligned16(X) || !aligned16(Y)) return fail(MQ_ERR_INVALID_ARG, "X and Y must be 16-byte aligned");
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
+    if (dev != w->device)
+        return fail(MQ_ERR_INVALID_ARG, "the current device is not the device that packed the weight");
+    if (next->device != w->device)
+        return fail(MQ_ERR_INVALID_ARG, "the next weight lives on another device");
+    L2Prefetch pf;
+    pf.p[0] = next->d.qweight;
+    pf.bytes[0] = next->d.N * next->d.K / 2;
+    pf.p[1] = next->d.sz;
+    pf.bytes[1] = next->d.N * next->d.Gp * 4;
+    return launch_decode(w, X, static_cast<int>(M), Y, reinterpret_cast<cudaStream_t>(stream), nullptr, pf);
 }
 
 mq_status mq_quantize_activations(const void *X, int64_t M, int64_t K, void *codes, float *scales,

@@ -7,6 +7,8 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "kernels.h"
+
 namespace mq {
 
 // Error codes a kernel leaves in the handle's device error word.
@@ -148,6 +150,28 @@ __device__ __forceinline__ uint32_t ldg_nc(const uint32_t *p) {
     uint32_t v;
     asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
+}
+
+// ---------------------------------------------------------------- L2 prefetch
+// Share `part` of `parts` of each region of pf, requested into L2 with bulk
+// prefetches (asynchronous, nothing waits for them).
+__device__ __forceinline__ void l2_prefetch_share(const L2Prefetch &pf, int part, int parts) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const long long bytes = pf.bytes[r];
+        if (bytes <= 0) continue;
+        const long long chunk = ((bytes + parts - 1) / parts + 15) & ~15ll;
+        const long long off = part * chunk;
+        if (off >= bytes) continue;
+        long long n = bytes - off < chunk ? bytes - off : chunk;
+        const char *ptr = static_cast<const char *>(pf.p[r]) + off;
+        while (n > 0) {
+            const unsigned piece = static_cast<unsigned>(n < (1ll << 20) ? n : (1ll << 20));
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(piece) : "memory");
+            ptr += piece;
+            n -= piece;
+        }
+    }
 }
 
 // ---------------------------------------------------------------- cp.async, clusters, PDL

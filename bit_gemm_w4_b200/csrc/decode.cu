@@ -62,6 +62,7 @@ struct DecodeParams {
     int M, N, K, G, Gp;
     int csr_cap;  // residual entries staged in shared memory (0: read from global)
     int with_residual;
+    L2Prefetch pf;  // the next layer's weight, brought into L2 meanwhile
 };
 
 template <int MX, int RT, int S, int BG, int CS>
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(Cfg<MX, RT, S, BG, CS>::THREADS)
     };
     Batch<BG> A, B;
     if (nb > 0) load(A, 0);
+    if (threadIdx.x == 0 && crank == 0) l2_prefetch_share(p.pf, tile, static_cast<int>(gridDim.x) / CS);
     pdl_launch_dependents();
 
     // ---------------------------------------------- stage X and the CSR slice
@@ -358,7 +360,7 @@ __global__ void __launch_bounds__(Cfg<MX, RT, S, BG, CS>::THREADS)
 
 template <int MX, int RT, int S, int BG, int CS>
 mq_status run(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t stream,
-              float *partial) {
+              float *partial, const L2Prefetch &pf) {
     using C = Cfg<MX, RT, S, BG, CS>;
     const DeviceWeight &d = weight_device(w);
     const bool with_residual = partial == nullptr;
@@ -384,6 +386,7 @@ mq_status run(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t st
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
     p.with_residual = with_residual ? 1 : 0;
+    p.pf = pf;
     // The tile's CSR slice is staged in shared memory while that keeps two
     // CTAs per SM; a longer slice (a dense or block-allocated residual) is
     // read from global memory by the walk instead.
@@ -439,26 +442,29 @@ int k_split(int M, int64_t K) {
 
 template <int MX, int RT, int S, int BG>
 mq_status run_cs(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t stream,
-                 float *partial) {
+                 float *partial, const L2Prefetch &pf) {
     switch (k_split(M, weight_device(w).K)) {
-        case 1: return run<MX, RT, S, BG, 1>(w, X, M, Y, stream, partial);
-        case 2: return run<MX, RT, S, BG, 2>(w, X, M, Y, stream, partial);
-        case 4: return run<MX, RT, S, BG, 4>(w, X, M, Y, stream, partial);
-        default: return run<MX, RT, S, BG, 8>(w, X, M, Y, stream, partial);
+        case 1: return run<MX, RT, S, BG, 1>(w, X, M, Y, stream, partial, pf);
+        case 2: return run<MX, RT, S, BG, 2>(w, X, M, Y, stream, partial, pf);
+        case 4: return run<MX, RT, S, BG, 4>(w, X, M, Y, stream, partial, pf);
+        default: return run<MX, RT, S, BG, 8>(w, X, M, Y, stream, partial, pf);
     }
 }
 
 }  // namespace
 
 mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t stream,
-                        float *partial) {
+                        float *partial, const L2Prefetch &pf) {
     if (M > 8) {
-        const mq_status st = launch_decode_wide(w, X, M, Y, stream, partial);
+        const mq_status st = launch_decode_wide(w, X, M, Y, stream, partial, pf);
         if (st != MQ_ERR_UNSUPPORTED) return st;
     }
-    if (M == 1) return run_cs<1, 1, 8, 4>(w, X, M, Y, stream, partial);
-    if (M <= 8) return run_cs<8, 2, 4, 2>(w, X, M, Y, stream, partial);
-    return run_cs<16, 4, 2, 2>(w, X, M, Y, stream, partial);
+    if (M == 1) return run_cs<1, 1, 8, 4>(w, X, M, Y, stream, partial, pf);
+    if (M <= 8) return run_cs<8, 2, 4, 2>(w, X, M, Y, stream, partial, pf);
+    const mq_status st = run_cs<16, 4, 2, 2>(w, X, M, Y, stream, partial, pf);
+    // X's slice of a very long K does not fit: the wide kernel streams X
+    if (st == MQ_ERR_UNSUPPORTED) return launch_decode_wide(w, X, M, Y, stream, partial, pf, true);
+    return st;
 }
 
 }  // namespace mq

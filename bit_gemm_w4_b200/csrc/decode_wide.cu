@@ -80,6 +80,7 @@ struct WideParams {
     int S;           // stages over all of K
     int ent_bytes;   // residual entry bytes of one slot; 0 = no residual
     int slot_bytes;  // bytes of one ring slot
+    L2Prefetch pf;   // the next layer's weight, brought into L2 meanwhile
 };
 
 // Bytes in front of the ring: the CTA's slice-start table, copied in 16-byte
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     for (int i = 0; i < NS - 1; ++i)
         if (i < nj) issue_weights(i);
+    if (threadIdx.x == 0) l2_prefetch_share(p.pf, blk, static_cast<int>(gridDim.x));
     pdl_launch_dependents();
     if (with_res) {
         cp_async_wait_group<0>();  // the table only: the copies above are not committed yet
@@ -374,7 +376,8 @@ mq_status run(const WideParams &p, int smem, int blocks, cudaStream_t stream) {
 }  // namespace
 
 mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
-                             cudaStream_t stream, float *partial) {
+                             cudaStream_t stream, float *partial, const L2Prefetch &pf,
+                             bool force) {
     if (M <= 8 || M > kMX) return MQ_ERR_UNSUPPORTED;
     const DeviceWeight &d = weight_device(w);
     const bool with_res = partial == nullptr && d.nnz > 0;
@@ -394,8 +397,9 @@ mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
     p.S = static_cast<int>((d.K + kKC - 1) / kKC);
+    p.pf = pf;
     const int64_t blocks = (d.N + kBN - 1) / kBN;
-    if (blocks < sm_count()) return MQ_ERR_UNSUPPORTED;  // the narrow kernel serves small layers
+    if (blocks < sm_count() && !force) return MQ_ERR_UNSUPPORTED;  // the narrow kernel serves small layers
     p.ent_bytes = with_res ? static_cast<int>(((d.wide_max + 15) / 8 + 1) * 16) : 0;
     if (with_res && (!d.wide_ptr || !d.wide_off || !d.wide_ent)) return MQ_ERR_UNSUPPORTED;
     const int raw = kXBytes + kWBytes + kSZBytes + (with_res ? kOffBytes + p.ent_bytes : 0);

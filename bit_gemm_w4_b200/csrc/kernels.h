@@ -75,18 +75,30 @@ const DeviceWeight &weight_device(const mq_weight *w);
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count();
 
+// Up to two regions of another weight (the next layer's packed codes and
+// scale words) that a decode launch brings into L2 while it runs: each CTA
+// issues one bulk L2 prefetch of its share. Addresses 16-byte aligned,
+// sizes multiples of 16; a size of 0 skips a region.
+struct L2Prefetch {
+    const void *p[2] = {nullptr, nullptr};
+    long long bytes[2] = {0, 0};
+};
+
 // Decode kernels (decode.cu): M in [1, 16]. With `partial` set the residual
 // is skipped and the dense base alone is written as fp32 to `partial`
 // (the unfused path's first half); else Y (bf16) gets the fused result.
 mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t stream,
-                        float *partial = nullptr);
+                        float *partial = nullptr, const L2Prefetch &pf = L2Prefetch());
 
 // Wide decode kernel (decode_wide.cu) for 8 < M <= 16; `partial` as for
 // decode. Returns MQ_ERR_UNSUPPORTED (without setting an error message) when
 // its stage ring cannot hold a residual slice, and the caller falls back to
 // launch_decode.
+// `force` also takes layers whose blocks do not fill the GPU (the fallback
+// when the narrow kernel cannot hold X's slice of a very long K).
 mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
-                             cudaStream_t stream, float *partial = nullptr);
+                             cudaStream_t stream, float *partial = nullptr,
+                             const L2Prefetch &pf = L2Prefetch(), bool force = false);
 
 // Prefill kernel (prefill.cu): any M >= 1; `partial` as for decode.
 mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,

@@ -62,6 +62,7 @@ def _load():
         "mq_pack": ([vp, i64, i64, ctypes.POINTER(_PackOpts), vp, ctypes.POINTER(vp)], st),
         "mq_linear": ([vp, vp, i64, vp, vp], st),
         "mq_linear_path": ([vp, vp, i64, vp, vp, ctypes.c_int], st),
+        "mq_linear_prefetch": ([vp, vp, i64, vp, vp, vp], st),
         "mq_linear_unfused": ([vp, vp, i64, vp, vp, ctypes.c_size_t, vp], st),
         "mq_linear_unfused_noalloc": ([vp, vp, i64, vp, vp], st),
         "mq_quantize_activations": ([vp, i64, i64, vp, vp, vp], st),
@@ -227,7 +228,14 @@ class Weight:
         self.linear_raw(X.data_ptr(), X.shape[0], Y.data_ptr(), stream=stream, path=path)
         return Y
 
-    def linear_raw(self, x_ptr: int, M: int, y_ptr: int, *, stream=None, path: str = "auto"):
+    def linear_raw(self, x_ptr: int, M: int, y_ptr: int, *, stream=None, path: str = "auto",
+                   next_weight: "Weight | None" = None):
+        """mq_linear on raw device pointers; with next_weight (decode only),
+        mq_linear_prefetch: that weight is brought into L2 meanwhile."""
+        if next_weight is not None and path == "auto":
+            _check(_lib.mq_linear_prefetch(self._h, x_ptr, M, y_ptr, next_weight._h,
+                                           _stream(stream)), "mq_linear_prefetch")
+            return
         _check(_lib.mq_linear_path(self._h, x_ptr, M, y_ptr, _stream(stream), _PATHS[path]),
                "mq_linear")
 

@@ -143,7 +143,21 @@ mq_status mq_pack(const float *W_host, int64_t N, int64_t K,
 mq_status mq_linear(const mq_weight *w, const void *X_dev, int64_t M,
                     void *Y_dev, mq_stream stream);
 
-/* As mq_linear with an explicit kernel choice. UNSUPPORTED for
+/* mq_linear, and while it runs, the packed codes and scale words of `next`
+ * (the layer that follows on this stream) are requested into the GPU's L2
+ * cache: each CTA of the decode kernel issues one bulk L2 prefetch of its
+ * share. A decode launch of one layer leaves most of the HBM bandwidth idle
+ * (it waits on latency), so the next layer's weights arrive meanwhile and
+ * its own launch reads them from L2. The result is that of mq_linear; `next`
+ * is only read. For M > 16, or next = NULL, this is mq_linear.
+ * Errors as mq_linear, plus INVALID_ARG when `next` lives on another
+ * device. */
+mq_status mq_linear_prefetch(const mq_weight *w, const void *X_dev, int64_t M, void *Y_dev,
+                             const mq_weight *next, mq_stream stream);
+
+/* As mq_linear with an explicit kernel choice (mq_linear: the decode
+ * kernels for M <= 16 unless X's slice of a very long K exceeds their shared
+ * memory, the prefill kernel otherwise). UNSUPPORTED for
  * MQ_PATH_DECODE with M > 16. */
 mq_status mq_linear_path(const mq_weight *w, const void *X_dev, int64_t M,
                          void *Y_dev, mq_stream stream, mq_path path);

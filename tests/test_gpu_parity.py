@@ -318,3 +318,30 @@ def test_wide_decode_ragged(mq, cuda, M):
     torch.cuda.synchronize()
     r = oracle_check(Yu, X, d)
     assert r["ok"], r
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_linear_prefetch_matches_linear(mq, cuda, M):
+    # bringing the next layer's weight into L2 changes nothing in the result
+    W1 = synth.weight(384, 4096, std=0.02, outlier_frac=0.005, seed=95)
+    W2 = synth.weight(1024, 384, std=0.02, outlier_frac=0.005, seed=96)
+    w1, w2 = mq.Weight.pack(W1, 0.01), mq.Weight.pack(W2, 0.01)
+    X = synth.activations(M, 4096, seed=97).cuda()
+    Y0 = w1.linear(X)
+    Y1 = torch.empty_like(Y0)
+    w1.linear_raw(X.data_ptr(), M, Y1.data_ptr(), next_weight=w2)
+    torch.cuda.synchronize()
+    assert torch.equal(Y0, Y1)
+    assert w1.device_error() == 0
+
+
+@pytest.mark.parametrize("M", [1, 8, 16])
+def test_longest_k_decode(mq, cuda, M):
+    # K = 65536 (the u16 column limit): at 16 tokens X's slice no longer fits
+    # the narrow kernel even split over 8 CTAs, and the wide kernel takes it
+    N, K = 64, 65536
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=98)
+    X = synth.activations(M, K, seed=99, channels=4, mult=20.0)
+    w, Y = _run(mq, W, X, 0.002)
+    r = oracle_check(Y, X, oracle.decompose(W, 0.002))
+    assert r["ok"], r
