@@ -295,18 +295,26 @@ def time_e2e(torch, ds: DecodeSet, steps: int, stream, dist_ctx):
 
 
 class DistCtx:
-    def __init__(self, torch):
+    """The replicas' plumbing: one process per GPU (RANK / LOCAL_RANK /
+    WORLD_SIZE from the launcher), a barrier around the timed region and the
+    maximum of the ranks' times. No data-path collective exists: the ranks
+    run independent replicas. backend "gloo" runs the same plumbing on CPU."""
+
+    def __init__(self, torch, backend: str = "nccl", timeout_s: int = 120):
         self.torch = torch
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = "cuda" if backend == "nccl" else "cpu"
         self.pg = None
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {}
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = torch.device("cuda", self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
             self.pg = dist
 
     def barrier(self):
@@ -316,13 +324,19 @@ class DistCtx:
     def max(self, v: float) -> float:
         if not self.pg:
             return v
-        t = self.torch.tensor([v], dtype=self.torch.float64, device="cuda")
+        t = self.torch.tensor([v], dtype=self.torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def job_throughput(step_bytes: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job TB/s: the bytes every replica processed over the slowest
+    rank's time (weak scaling: each rank runs the full step)."""
+    return step_bytes * steps * world / (ms_max * 1e-3) / 1e12
 
 
 def secondary(torch, mq, dev, stream, pk, which: str, reps: int):
@@ -378,10 +392,10 @@ def run_ours(args):
                                   dist_ctx, dist_ctx.local)
     per_shape = time_per_shape(torch, ds, stream)
     step_bytes = sum(ds.bytes_per_launch)
-    value = step_bytes * args.steps * dist_ctx.world / (ms * 1e-3) / 1e12
+    value = job_throughput(step_bytes, args.steps, dist_ctx.world, ms)
     e2e_steps = min(args.steps, 500)
     ms_e2e, h2d, d2h = time_e2e(torch, ds, e2e_steps, stream, dist_ctx)
-    e2e = step_bytes * e2e_steps * dist_ctx.world / (ms_e2e * 1e-3) / 1e12
+    e2e = job_throughput(step_bytes, e2e_steps, dist_ctx.world, ms_e2e)
     # the fused decode kernel is the only kernel of a step: its achieved
     # bandwidth is the step's algorithmic bytes over the step's device time
     achieved = step_bytes * args.steps / (ms * 1e-3) / 1e9
