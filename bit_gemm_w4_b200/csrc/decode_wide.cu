@@ -87,7 +87,8 @@ struct WideParams {
 // chunks from a 4-entry-aligned start, then one residual fragment tile per
 // warp.
 __host__ __device__ constexpr int wtab_bytes(int spr) { return ((spr + 8) / 4 + 1) * 16; }
-constexpr int kTileBytes = 512;  // 16 rows x 16 k-slots of bf16, A-fragment order
+constexpr int kFrag = 512;               // 16 rows x 16 k-slots of bf16, A-fragment order
+constexpr int kTileBytes = 4 * kFrag;    // the fragments of four k-steps
 __host__ __device__ constexpr int ring_offset(int spr) { return wtab_bytes(spr) + kWarps * kTileBytes; }
 
 // Byte offset in a fragment tile of the code at row r (0..15), column c of a
@@ -200,7 +201,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) racc[nt][i] = 0.f;
-    sts128(rtile + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) sts128(rtile + u * kFrag + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
     __syncwarp();
 
     for (int i = 0; i < nj; ++i) {
@@ -276,7 +278,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 acc[nt][2] = fmaf(s1, c[nt][2], acc[nt][2]);
                 acc[nt][3] = fmaf(s1, c[nt][3], acc[nt][3]);
             }
-            // sparse branch: the warp's entries of this group, k-step by k-step
+            // sparse branch: the warp's entries of this group, four k-steps per
+            // scatter; k-steps without entries issue no MMA
             if (with_res) {
                 const uint16_t *offw =
                     reinterpret_cast<const uint16_t *>(sl + kXBytes + kWBytes + kSZBytes) +
@@ -284,28 +287,36 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const uint16_t *ent = reinterpret_cast<const uint16_t *>(
                                           sl + kXBytes + kWBytes + kSZBytes + kOffBytes) +
                                       (wtab[blk * p.S + j - kbase] & 7);
-                int a = lds_u16(offw);
+                int o[9];
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const int b = lds_u16(offw + ks + 1);
-                    if (b > a) {  // the same for every lane
-                        for (int e = a + lane; e < b; e += 32) {
+                for (int i = 0; i < 9; ++i) o[i] = static_cast<int>(lds_u16(offw + i));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (o[4 * h + 4] > o[4 * h]) {  // the same for every lane
+                        for (int e = o[4 * h] + lane; e < o[4 * h + 4]; e += 32) {
                             const uint32_t v = lds_u16(ent + e);
+                            const int c = static_cast<int>(v & 0x7Fu);
                             const int q = static_cast<int>(((v >> 12) & 0xFu) ^ 8u) - 8;
-                            sts_u16(rtile + tile_pos(static_cast<int>((v >> 8) & 0xFu),
-                                                     static_cast<int>(v & 0x7Fu)),
+                            sts_u16(rtile + (((c & 31) >> 2) & 3) * kFrag +
+                                        tile_pos(static_cast<int>((v >> 8) & 0xFu), c),
                                     __float_as_uint(static_cast<float>(q)) >> 16);
                         }
                         __syncwarp();
-                        const uint4 f = lds128(rtile + 16 * lane);
-                        sts128(rtile + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
-                        __syncwarp();
-                        const uint32_t fa[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-                        for (int nt = 0; nt < 2; ++nt)
-                            mma_bf16_16816(racc[nt], fa, xb[nt][2 * ks], xb[nt][2 * ks + 1], racc[nt]);
+                        for (int u = 0; u < 4; ++u) {
+                            const int ks = 4 * h + u;
+                            if (o[ks + 1] > o[ks]) {
+                                const uint4 f = lds128(rtile + u * kFrag + 16 * lane);
+                                sts128(rtile + u * kFrag + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
+                                const uint32_t fa[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                                for (int nt = 0; nt < 2; ++nt)
+                                    mma_bf16_16816(racc[nt], fa, xb[nt][2 * ks], xb[nt][2 * ks + 1],
+                                                   racc[nt]);
+                            }
+                        }
+                        __syncwarp();
                     }
-                    a = b;
                 }
             }
         }
