@@ -27,12 +27,9 @@ struct mq_weight {
     std::vector<void *> allocations;
     std::vector<int32_t> host_row_ptr;  // for residual tile statistics
     mutable std::mutex maps_mu;
-    mutable std::vector<mq::MapSet *> maps;
+    mutable std::vector<std::pair<int, int64_t>> tile_nnz;  // (tile height, max entries)
     mutable mq::PrefillMaps *pmaps = nullptr;
-    ~mq_weight() {
-        for (auto *m : maps) delete m;
-        delete pmaps;
-    }
+    ~mq_weight() { delete pmaps; }
 };
 
 namespace mq {
@@ -52,20 +49,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
     });
     return fn;
-}
-
-bool encode_2d_u32(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
-                   uint32_t box_inner, uint32_t box_outer) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {inner * 4};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
 }
 
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, int esize, const void *base,
@@ -271,28 +254,17 @@ int sm_count() {
     return sms[dev];
 }
 
-const MapSet *weight_maps(const mq_weight *w, int bn, int gs) {
+int64_t max_tile_nnz(const mq_weight *w, int bn) {
     std::lock_guard<std::mutex> lock(w->maps_mu);
-    for (auto *m : w->maps)
-        if (m->bn == bn && m->gs == gs) return m;
-    MapSet *m = new (std::nothrow) MapSet();
-    if (!m) return nullptr;
-    m->bn = bn;
-    m->gs = gs;
-    const DeviceWeight &d = w->d;
-    if (!encode_2d_u32(&m->w, d.qweight, d.K / 8, d.N, 16, bn) ||
-        !encode_2d_u32(&m->sz, d.sz, d.Gp, d.N, gs, bn)) {
-        delete m;
-        fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-        return nullptr;
+    for (const auto &e : w->tile_nnz)
+        if (e.first == bn) return e.second;
+    int64_t mx = 0;
+    for (int64_t r = 0; r < w->d.N; r += bn) {
+        const int64_t r1 = std::min<int64_t>(w->d.N, r + bn);
+        mx = std::max<int64_t>(mx, w->host_row_ptr[r1] - w->host_row_ptr[r]);
     }
-    for (int64_t r = 0; r < d.N; r += bn) {
-        int64_t r1 = std::min<int64_t>(d.N, r + bn);
-        m->max_tile_nnz = std::max<int64_t>(m->max_tile_nnz,
-                                            w->host_row_ptr[r1] - w->host_row_ptr[r]);
-    }
-    w->maps.push_back(m);
-    return m;
+    w->tile_nnz.emplace_back(bn, mx);
+    return mx;
 }
 
 const PrefillMaps *prefill_maps(const mq_weight *w) {

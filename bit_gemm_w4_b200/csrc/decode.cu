@@ -364,12 +364,7 @@ mq_status run(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t st
     using C = Cfg<MX, RT, S, BG, CS>;
     const DeviceWeight &d = weight_device(w);
     const bool with_residual = partial == nullptr;
-    int64_t tile_nnz = 0;
-    if (with_residual) {
-        const MapSet *maps = weight_maps(w, C::BN, 4);
-        if (!maps) return MQ_ERR_CUDA;
-        tile_nnz = maps->max_tile_nnz;
-    }
+    const int64_t tile_nnz = with_residual ? max_tile_nnz(w, C::BN) : 0;
     DecodeParams p;
     p.qweight = d.qweight;
     p.sz = d.sz;

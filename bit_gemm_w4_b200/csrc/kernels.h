@@ -48,17 +48,9 @@ struct DeviceWeight {
     int *err;                 // device error word
 };
 
-// Tensor maps and residual-slice sizes a kernel configuration needs; filled
-// by the host at pack time (see api.cpp).
-struct MapSet {
-    int bn = 0, gs = 0;
-    CUtensorMap w;   // qweight, box [bn rows][16 words]
-    CUtensorMap sz;  // sz, box [bn rows][gs words]
-    int64_t max_tile_nnz = 0;  // max residual entries over bn-row tiles
-};
-
-// Looks up (or builds) the MapSet for a tile shape of a handle.
-const MapSet *weight_maps(const mq_weight *w, int bn, int gs);
+// Largest residual entry count over the bn-row tiles of a handle (cached per
+// tile height; the decode kernels size their shared-memory CSR slice with it).
+int64_t max_tile_nnz(const mq_weight *w, int bn);
 
 // Tensor maps of the prefill kernel (built once per handle).
 struct PrefillMaps {

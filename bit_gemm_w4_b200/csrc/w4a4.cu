@@ -437,12 +437,7 @@ mq_status run_a4(const mq_weight *w, const int8_t *codes, const float *xscale, i
                  cudaStream_t stream) {
     using C = A4Cfg<MX, RT, S, BG, CS>;
     const DeviceWeight &d = weight_device(w);
-    int64_t tile_nnz = 0;
-    if (d.nnz > 0) {
-        const MapSet *maps = weight_maps(w, C::BN, 4);
-        if (!maps) return MQ_ERR_CUDA;
-        tile_nnz = maps->max_tile_nnz;
-    }
+    const int64_t tile_nnz = d.nnz > 0 ? max_tile_nnz(w, C::BN) : 0;
     A4Params p;
     p.qweight = d.qweight;
     p.sz = d.sz;
