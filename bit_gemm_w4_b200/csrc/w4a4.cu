@@ -505,7 +505,13 @@ mq_status launch_quantize(const void *X, int64_t M, int64_t K, void *codes, floa
 
 mq_status launch_decode_a4(const mq_weight *w, const int8_t *codes, const float *xscale, int M,
                            void *Y, cudaStream_t stream) {
-    if (M == 1) return run_a4_cs<8, 1, 8, 4>(w, codes, xscale, M, Y, stream);
+    if (M == 1) {
+        // as for the W4A16 kernel: 4-warp CTAs when the 16-row tiles exceed
+        // two 8-warp CTAs per SM
+        if ((weight_device(w).N + 15) / 16 > 2 * static_cast<int64_t>(sm_count()))
+            return run_a4_cs<8, 1, 4, 4>(w, codes, xscale, M, Y, stream);
+        return run_a4_cs<8, 1, 8, 4>(w, codes, xscale, M, Y, stream);
+    }
     if (M <= 8) return run_a4_cs<8, 2, 4, 2>(w, codes, xscale, M, Y, stream);
     return run_a4_cs<16, 4, 2, 2>(w, codes, xscale, M, Y, stream);
 }
