@@ -533,7 +533,7 @@ mq_status mq_quantize_activations(const void *X, int64_t M, int64_t K, void *cod
     if (!X || !codes || !scales) return fail(MQ_ERR_INVALID_ARG, "X, codes or scales is NULL");
     if (!aligned16(X) || !aligned16(codes) || !aligned16(scales))
         return fail(MQ_ERR_INVALID_ARG, "X, codes and scales must be 16-byte aligned");
-    return launch_quantize(X, M, K, codes, scales, reinterpret_cast<cudaStream_t>(stream));
+    return launch_quantize(X, M, K, codes, scales, reinterpret_cast<cudaStream_t>(stream), false);
 }
 
 int64_t mq_w4a4_workspace_bytes(const mq_weight *w, int64_t M) {
@@ -560,7 +560,7 @@ mq_status mq_linear_w4a4(const mq_weight *w, const void *X, int64_t M, void *Y, 
     int8_t *codes = static_cast<int8_t *>(workspace);
     float *scales = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                               (M * w->d.K + 15) / 16 * 16);
-    mq_status st = launch_quantize(X, M, w->d.K, codes, scales, s);
+    mq_status st = launch_quantize(X, M, w->d.K, codes, scales, s, true);
     if (st) return st;
     return launch_decode_a4(w, codes, scales, static_cast<int>(M), Y, s);
 }

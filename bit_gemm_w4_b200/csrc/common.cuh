@@ -267,6 +267,22 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
           "f"(c[2]), "f"(c[3]));
 }
 
+// D = A * B + C, m16n8k32, s8 inputs, s32 accumulate (exact).
+__device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Four int8 bytes q - z from four nibbles 0..15 held in the low half of each
+// byte of v: (v | 0x80) - z never borrows across bytes; ^ 0x80 restores sign.
+__device__ __forceinline__ uint32_t codes_minus_zero(uint32_t nib4, uint32_t zz4) {
+    return ((nib4 | 0x80808080u) - zz4) ^ 0x80808080u;
+}
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) {
     return __uint_as_float(b16 << 16);
 }
@@ -279,6 +295,10 @@ __device__ __forceinline__ uint32_t lds_u16(const void *p) {
     unsigned short v;
     asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_u32(p)));
     return v;
+}
+
+__device__ __forceinline__ void sts_u8(void *p, uint32_t v) {
+    asm volatile("st.shared.u8 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void sts_u16(void *p, uint32_t v) {

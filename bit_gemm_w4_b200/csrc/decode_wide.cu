@@ -44,8 +44,15 @@
 // Launches use programmatic dependent launch: codes, scales and residual
 // entries (which no earlier kernel writes) are requested before
 // griddepcontrol.wait; X is read and Y written only after it.
+//
+// The same ring serves the W4A4 variant (A4 = true): a slot then holds the
+// int8 activation codes of the stage (each 8-column chunk's bytes already in
+// the packed codes' k order), the dense branch turns nibbles into int8 q - z
+// and sums each group exactly with mma.sync m16n8k32 s8, the residual
+// k-steps become int8 fragments, and Y = s_x * (sum_g s_g D_g + s_r R).
 
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -59,17 +66,22 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kBN = 16 * kWarps;             // rows per CTA
 constexpr int kKC = 256;                     // columns per stage (two groups)
 constexpr int kMX = 16;                      // token capacity
-constexpr int kXRS = kKC * 2 + 16;           // X row stride in a slot (bytes)
-constexpr int kXBytes = kMX * kXRS;          // 8448
 constexpr int kWBytes = kBN * (kKC / 2);     // [warp][group][16 rows][64 B]
 constexpr int kSZBytes = kBN * 2 * 4;        // [warp][group][16 rows] u32
 constexpr int kOffBytes = kWideOffStride * 2;
+// A slot: codes, scale words, residual offsets, residual entries, then X.
+constexpr int kSZOff = kWBytes, kOffOff = kSZOff + kSZBytes, kEntOff = kOffOff + kOffBytes;
+// X row stride in a slot (bytes): bf16, or int8 codes (W4A4)
+template <bool A4>
+__host__ __device__ constexpr int x_row_stride() { return A4 ? kKC + 16 : kKC * 2 + 16; }
 constexpr int kSmemLimit = 112 * 1024;       // two CTAs per SM
 
 struct WideParams {
     const uint32_t *qweight;  // [N][K/8]
     const uint32_t *sz;       // [N][Gp]
     const __nv_bfloat16 *X;   // [M][K]
+    const int8_t *codes;      // [M][K] activation codes (W4A4), chunk bytes permuted
+    const float *xscale;      // [M] activation scales (W4A4)
     __nv_bfloat16 *Y;         // [M][N]
     float *Yf;                // fp32 dense-only output (unfused path) or null
     const int32_t *wptr;
@@ -79,6 +91,7 @@ struct WideParams {
     int M, N, K, G, Gp;
     int S;           // stages over all of K
     int ent_bytes;   // residual entry bytes of one slot; 0 = no residual
+    int x_off;       // X's offset in a slot (kEntOff + ent_bytes)
     int slot_bytes;  // bytes of one ring slot
     L2Prefetch pf;   // the next layer's weight, brought into L2 meanwhile
 };
@@ -99,11 +112,21 @@ __device__ __forceinline__ int tile_pos(int r, int c) {
     return (((r & 7) * 4 + (c >> 5)) * 4 + (r >> 3) + 2 * ((c & 3) >> 1)) * 4 + (c & 1) * 2;
 }
 
+// The same for the int8 m16n8k32 A layout (W4A4): column c of a group sits
+// at byte ((c & 3) << 1) | ((c >> 2) & 1) of its 8-column chunk in the
+// packed codes' k order; positions 0..3 go to registers (r / 8), 4..7 to
+// 2 + (r / 8), of thread (g = r % 8, t = c / 32); k-step (c % 32) / 8.
+__device__ __forceinline__ int tile_pos_a4(int r, int c) {
+    const int pos = ((c & 3) << 1) | ((c >> 2) & 1);
+    return ((r & 7) * 4 + (c >> 5)) * 16 + ((r >> 3) + ((pos >> 2) << 1)) * 4 + (pos & 3);
+}
+
 __device__ __forceinline__ int xchunk(int c) { return c ^ (((c >> 3) & 1) << 1); }
 
-template <int NS>
+template <bool A4, int NS>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_wide_kernel(const __grid_constant__ WideParams p) {
+    constexpr int XRS = x_row_stride<A4>();
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -135,36 +158,43 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int jj = 0; jj < 2; ++jj) {
             const int gi = 2 * j + jj;
             if (gi < G) {
-                uint8_t *wd = sl + kXBytes + (warp * 2 + jj) * 16 * 64 + 16 * t;
+                uint8_t *wd = sl + (warp * 2 + jj) * 16 * 64 + 16 * t;
                 cp_async16(wd + g * 64, w0 + gi * 16);
                 cp_async16(wd + (g + 8) * 64, w1 + gi * 16);
             }
         }
         if (2 * j + zj < G)
-            cp_async4(sl + kXBytes + kWBytes + ((warp * 2 + zj) * 16 + zrow) * 4, szp + 2 * j);
+            cp_async4(sl + kSZOff + ((warp * 2 + zj) * 16 + zrow) * 4, szp + 2 * j);
     };
     auto issue_residual = [&](int i) {
         uint8_t *sl = slot_of(i);
         const int key = blk * p.S + j_lo + i;
         if (threadIdx.x < kOffBytes / 16)
-            cp_async16(sl + kXBytes + kWBytes + kSZBytes + 16 * threadIdx.x,
+            cp_async16(sl + kOffOff + 16 * threadIdx.x,
                        p.woff + static_cast<size_t>(key) * kWideOffStride + 8 * threadIdx.x);
         const int eb = wtab[key - kbase], ee = wtab[key - kbase + 1];
         const int base = eb & ~7, n16 = (ee - base + 7) >> 3;
-        uint8_t *ed = sl + kXBytes + kWBytes + kSZBytes + kOffBytes;
+        uint8_t *ed = sl + kEntOff;
         for (int c = threadIdx.x; c < n16; c += kThreads) cp_async16(ed + 16 * c, p.went + base + 8 * c);
     };
     auto issue_x = [&](int i) {
-        uint8_t *sl = slot_of(i);
+        uint8_t *sx = slot_of(i) + p.x_off;
         const int k0 = (j_lo + i) * kKC;
-        const int chunks = min(kKC, K - k0) / 8;
+        if constexpr (A4) {
+            // 16 chunks of 16 codes per token row, one per thread
+            const int tok = threadIdx.x >> 4, c = threadIdx.x & 15;
+            if (tok < M && 16 * c < K - k0)
+                cp_async16(sx + tok * XRS + 16 * c, p.codes + static_cast<size_t>(tok) * K + k0 + 16 * c);
+        } else {
+            const int chunks = min(kKC, K - k0) / 8;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int idx = threadIdx.x + kThreads * u;
-            const int tok = idx >> 5, c = idx & 31;
-            if (tok < M && c < chunks)
-                cp_async16(sl + tok * kXRS + xchunk(c) * 16,
-                           p.X + static_cast<size_t>(tok) * K + k0 + 8 * c);
+            for (int u = 0; u < 2; ++u) {
+                const int idx = threadIdx.x + kThreads * u;
+                const int tok = idx >> 5, c = idx & 31;
+                if (tok < M && c < chunks)
+                    cp_async16(sx + tok * XRS + xchunk(c) * 16,
+                               p.X + static_cast<size_t>(tok) * K + k0 + 8 * c);
+            }
         }
     };
 
@@ -196,11 +226,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-    float racc[2][4];  // sparse branch, in the accumulator layout of acc
+    // sparse branch, in the accumulator layout of acc (fp32 sums of exact
+    // bf16 products, or exact int32 sums for W4A4)
+    using RAcc = typename std::conditional<A4, int, float>::type;
+    RAcc racc[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) racc[nt][i] = 0.f;
+        for (int i = 0; i < 4; ++i) racc[nt][i] = 0;
 #pragma unroll
     for (int u = 0; u < 4; ++u) sts128(rtile + u * kFrag + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
     __syncwarp();
@@ -216,31 +249,35 @@ __global__ void __launch_bounds__(kThreads, 2)
         cp_async_commit();
 
         const uint8_t *sl = slot_of(i);
+        const uint8_t *sx = sl + p.x_off;
         const int j = j_lo + i;
-        // dense branch
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
             const int gi = 2 * j + jj;
             if (gi >= G) break;
-            const uint8_t *wd = sl + kXBytes + (warp * 2 + jj) * 16 * 64 + 16 * t;
+            // ---------------------------------------- dense branch
+            const uint8_t *wd = sl + (warp * 2 + jj) * 16 * 64 + 16 * t;
             const uint4 wa = lds128(wd + g * 64), wb = lds128(wd + (g + 8) * 64);
-            const uint32_t *zs =
-                reinterpret_cast<const uint32_t *>(sl + kXBytes + kWBytes) + (warp * 2 + jj) * 16;
+            const uint32_t *zs = reinterpret_cast<const uint32_t *>(sl + kSZOff) + (warp * 2 + jj) * 16;
             const uint32_t sz0 = zs[g], sz1 = zs[g + 8];
             const float s0 = half_bits_to_f32(sz0), s1 = half_bits_to_f32(sz1);
             const uint32_t z0 = static_cast<uint32_t>(half_bits_to_f32(sz0 >> 16));
             const uint32_t z1 = static_cast<uint32_t>(half_bits_to_f32(sz1 >> 16));
-            const uint32_t zz0 = (0x4300u | z0) * 0x00010001u;  // bf16x2 (128+z)
-            const uint32_t zz1 = (0x4300u | z1) * 0x00010001u;
-            uint32_t xb[2][16];
+            const uint32_t wr0[4] = {wa.x, wa.y, wa.z, wa.w};
+            const uint32_t wr1[4] = {wb.x, wb.y, wb.z, wb.w};
+            // X fragments of tokens g and g + 8 (16 words of bf16 pairs, or 8
+            // words of int8 codes)
+            constexpr int XW = A4 ? 8 : 16;
+            uint32_t xb[2][XW];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 const int tok = g + 8 * nt;
                 if (tok < M) {
-                    const uint8_t *xr = sl + tok * kXRS;
+                    const uint8_t *xr = sx + tok * XRS;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 v = lds128(xr + xchunk(16 * jj + 4 * t + q) * 16);
+                    for (int q = 0; q < XW / 4; ++q) {
+                        const uint4 v = A4 ? lds128(xr + jj * 128 + 32 * t + 16 * q)
+                                           : lds128(xr + xchunk(16 * jj + 4 * t + q) * 16);
                         xb[nt][4 * q + 0] = v.x;
                         xb[nt][4 * q + 1] = v.y;
                         xb[nt][4 * q + 2] = v.z;
@@ -248,71 +285,107 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) xb[nt][q] = 0u;
+                    for (int q = 0; q < XW; ++q) xb[nt][q] = 0u;
                 }
             }
-            float c[2][4];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) c[nt][q] = 0.f;
-            const uint32_t wr0[4] = {wa.x, wa.y, wa.z, wa.w};
-            const uint32_t wr1[4] = {wb.x, wb.y, wb.z, wb.w};
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t a_lo = wr0[ks >> 1] >> (8 * (ks & 1));
-                const uint32_t b_lo = wr1[ks >> 1] >> (8 * (ks & 1));
-                uint32_t a[4];
-                a[0] = bf16x2_sub(nib_pair_bias128(a_lo), zz0);
-                a[1] = bf16x2_sub(nib_pair_bias128(b_lo), zz1);
-                a[2] = bf16x2_sub(nib_pair_bias128(a_lo >> 4), zz0);
-                a[3] = bf16x2_sub(nib_pair_bias128(b_lo >> 4), zz1);
+            if constexpr (A4) {
+                const uint32_t zz0 = z0 * 0x01010101u, zz1 = z1 * 0x01010101u;
+                int d[2][4];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
-                    mma_bf16_16816(c[nt], a, xb[nt][2 * ks], xb[nt][2 * ks + 1], c[nt]);
-            }
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                acc[nt][0] = fmaf(s0, c[nt][0], acc[nt][0]);
-                acc[nt][1] = fmaf(s0, c[nt][1], acc[nt][1]);
-                acc[nt][2] = fmaf(s1, c[nt][2], acc[nt][2]);
-                acc[nt][3] = fmaf(s1, c[nt][3], acc[nt][3]);
+                    for (int q = 0; q < 4; ++q) d[nt][q] = 0;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint32_t a[4];
+                    a[0] = codes_minus_zero(wr0[ks] & 0x0F0F0F0Fu, zz0);
+                    a[1] = codes_minus_zero(wr1[ks] & 0x0F0F0F0Fu, zz1);
+                    a[2] = codes_minus_zero((wr0[ks] >> 4) & 0x0F0F0F0Fu, zz0);
+                    a[3] = codes_minus_zero((wr1[ks] >> 4) & 0x0F0F0F0Fu, zz1);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) mma_s8_16832(d[nt], a, xb[nt][2 * ks], xb[nt][2 * ks + 1]);
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    acc[nt][0] = fmaf(s0, static_cast<float>(d[nt][0]), acc[nt][0]);
+                    acc[nt][1] = fmaf(s0, static_cast<float>(d[nt][1]), acc[nt][1]);
+                    acc[nt][2] = fmaf(s1, static_cast<float>(d[nt][2]), acc[nt][2]);
+                    acc[nt][3] = fmaf(s1, static_cast<float>(d[nt][3]), acc[nt][3]);
+                }
+            } else {
+                const uint32_t zz0 = (0x4300u | z0) * 0x00010001u;  // bf16x2 (128+z)
+                const uint32_t zz1 = (0x4300u | z1) * 0x00010001u;
+                float c[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) c[nt][q] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t a_lo = wr0[ks >> 1] >> (8 * (ks & 1));
+                    const uint32_t b_lo = wr1[ks >> 1] >> (8 * (ks & 1));
+                    uint32_t a[4];
+                    a[0] = bf16x2_sub(nib_pair_bias128(a_lo), zz0);
+                    a[1] = bf16x2_sub(nib_pair_bias128(b_lo), zz1);
+                    a[2] = bf16x2_sub(nib_pair_bias128(a_lo >> 4), zz0);
+                    a[3] = bf16x2_sub(nib_pair_bias128(b_lo >> 4), zz1);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+                        mma_bf16_16816(c[nt], a, xb[nt][2 * ks], xb[nt][2 * ks + 1], c[nt]);
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    acc[nt][0] = fmaf(s0, c[nt][0], acc[nt][0]);
+                    acc[nt][1] = fmaf(s0, c[nt][1], acc[nt][1]);
+                    acc[nt][2] = fmaf(s1, c[nt][2], acc[nt][2]);
+                    acc[nt][3] = fmaf(s1, c[nt][3], acc[nt][3]);
+                }
             }
-            // sparse branch: the warp's entries of this group, four k-steps per
-            // scatter; k-steps without entries issue no MMA
+            // ---------------------------------------- sparse branch
+            // the warp's entries of this group, scattered into fragment tiles
+            // a half-group (four bf16 k-steps, two int8 k-steps) at a time;
+            // k-steps without entries issue no MMA
             if (with_res) {
                 const uint16_t *offw =
-                    reinterpret_cast<const uint16_t *>(sl + kXBytes + kWBytes + kSZBytes) +
-                    warp * 16 + jj * 8;
-                const uint16_t *ent = reinterpret_cast<const uint16_t *>(
-                                          sl + kXBytes + kWBytes + kSZBytes + kOffBytes) +
+                    reinterpret_cast<const uint16_t *>(sl + kOffOff) + warp * 16 + jj * 8;
+                const uint16_t *ent = reinterpret_cast<const uint16_t *>(sl + kEntOff) +
                                       (wtab[blk * p.S + j - kbase] & 7);
                 int o[9];
 #pragma unroll
-                for (int i = 0; i < 9; ++i) o[i] = static_cast<int>(lds_u16(offw + i));
+                for (int q = 0; q < 9; ++q) o[q] = static_cast<int>(lds_u16(offw + q));
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     if (o[4 * h + 4] > o[4 * h]) {  // the same for every lane
                         for (int e = o[4 * h] + lane; e < o[4 * h + 4]; e += 32) {
                             const uint32_t v = lds_u16(ent + e);
                             const int c = static_cast<int>(v & 0x7Fu);
+                            const int r = static_cast<int>((v >> 8) & 0xFu);
                             const int q = static_cast<int>(((v >> 12) & 0xFu) ^ 8u) - 8;
-                            sts_u16(rtile + (((c & 31) >> 2) & 3) * kFrag +
-                                        tile_pos(static_cast<int>((v >> 8) & 0xFu), c),
-                                    __float_as_uint(static_cast<float>(q)) >> 16);
+                            if constexpr (A4)
+                                sts_u8(rtile + ((c >> 3) & 1) * kFrag + tile_pos_a4(r, c),
+                                       static_cast<uint32_t>(q) & 0xFFu);
+                            else
+                                sts_u16(rtile + (((c & 31) >> 2) & 3) * kFrag + tile_pos(r, c),
+                                        __float_as_uint(static_cast<float>(q)) >> 16);
                         }
                         __syncwarp();
+                        constexpr int KPH = A4 ? 2 : 4;  // k-steps per half-group
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int ks = 4 * h + u;
-                            if (o[ks + 1] > o[ks]) {
+                        for (int u = 0; u < KPH; ++u) {
+                            const int ks = KPH * h + u;  // k-step of the group
+                            const int l0 = A4 ? 2 * ks : ks, l1 = A4 ? 2 * ks + 2 : ks + 1;
+                            if (o[l1] > o[l0]) {
                                 const uint4 f = lds128(rtile + u * kFrag + 16 * lane);
                                 sts128(rtile + u * kFrag + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
                                 const uint32_t fa[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-                                for (int nt = 0; nt < 2; ++nt)
-                                    mma_bf16_16816(racc[nt], fa, xb[nt][2 * ks], xb[nt][2 * ks + 1],
-                                                   racc[nt]);
+                                for (int nt = 0; nt < 2; ++nt) {
+                                    if constexpr (A4)
+                                        mma_s8_16832(racc[nt], fa, xb[nt][2 * ks], xb[nt][2 * ks + 1]);
+                                    else
+                                        mma_bf16_16816(racc[nt], fa, xb[nt][2 * ks],
+                                                       xb[nt][2 * ks + 1], racc[nt]);
+                                }
                             }
                         }
                         __syncwarp();
@@ -338,9 +411,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int i = 0; i < 4; ++i) {
             const int row = 16 * warp + g + ((i < 2) ? 0 : 8);
             const int tok = 8 * nt + 2 * t + (i & 1);
-            res[row * kMX + tok] = fmaf(i < 2 ? sra : srb, racc[nt][i], acc[nt][i]);
+            float y = fmaf(i < 2 ? sra : srb, static_cast<float>(racc[nt][i]), acc[nt][i]);
+            if constexpr (A4) y *= tok < M ? p.xscale[tok] : 0.f;
+            res[row * kMX + tok] = y;
         }
-
     __syncthreads();
     for (int idx = threadIdx.x; idx < M * kBN; idx += kThreads) {
         const int m = idx / kBN, r = idx % kBN, n = n0 + r;
@@ -354,9 +428,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-template <int NS>
+template <bool A4, int NS>
 mq_status run(const WideParams &p, int smem, int blocks, cudaStream_t stream) {
-    auto kern = decode_wide_kernel<NS>;
+    auto kern = decode_wide_kernel<A4, NS>;
     static bool configured[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
@@ -384,20 +458,15 @@ mq_status run(const WideParams &p, int smem, int blocks, cudaStream_t stream) {
     return MQ_OK;
 }
 
-}  // namespace
-
-mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
-                             cudaStream_t stream, float *partial, const L2Prefetch &pf,
-                             bool force) {
+// Fills the shared part of the parameters and picks the ring depth; returns
+// MQ_ERR_UNSUPPORTED (no message) when the kernel should not or cannot take
+// the call.
+template <bool A4>
+mq_status launch(WideParams &p, const DeviceWeight &d, int M, bool with_res, bool force,
+                 cudaStream_t stream) {
     if (M <= 8 || M > kMX) return MQ_ERR_UNSUPPORTED;
-    const DeviceWeight &d = weight_device(w);
-    const bool with_res = partial == nullptr && d.nnz > 0;
-    WideParams p;
     p.qweight = d.qweight;
     p.sz = d.sz;
-    p.X = static_cast<const __nv_bfloat16 *>(X);
-    p.Y = static_cast<__nv_bfloat16 *>(Y);
-    p.Yf = partial;
     p.wptr = d.wide_ptr;
     p.woff = d.wide_off;
     p.went = d.wide_ent;
@@ -408,22 +477,45 @@ mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
     p.S = static_cast<int>((d.K + kKC - 1) / kKC);
-    p.pf = pf;
     const int64_t blocks = (d.N + kBN - 1) / kBN;
-    if (blocks < sm_count() && !force) return MQ_ERR_UNSUPPORTED;  // the narrow kernel serves small layers
+    if (blocks < sm_count() && !force) return MQ_ERR_UNSUPPORTED;  // the narrow kernels serve small layers
     p.ent_bytes = with_res ? static_cast<int>(((d.wide_max + 15) / 8 + 1) * 16) : 0;
     if (with_res && (!d.wide_ptr || !d.wide_off || !d.wide_ent)) return MQ_ERR_UNSUPPORTED;
-    const int raw = kXBytes + kWBytes + kSZBytes + (with_res ? kOffBytes + p.ent_bytes : 0);
-    p.slot_bytes = (raw + 127) / 128 * 128;
+    p.x_off = kEntOff + p.ent_bytes;
+    p.slot_bytes = (p.x_off + kMX * x_row_stride<A4>() + 127) / 128 * 128;
     int ns = 4;
     while (ns >= 2 && ring_offset(p.S) + ns * p.slot_bytes > kSmemLimit) --ns;
     if (ns < 2) return MQ_ERR_UNSUPPORTED;  // a residual slice too long for the ring
     const int smem = ring_offset(p.S) + ns * p.slot_bytes;
     switch (ns) {
-        case 4: return run<4>(p, smem, static_cast<int>(blocks), stream);
-        case 3: return run<3>(p, smem, static_cast<int>(blocks), stream);
-        default: return run<2>(p, smem, static_cast<int>(blocks), stream);
+        case 4: return run<A4, 4>(p, smem, static_cast<int>(blocks), stream);
+        case 3: return run<A4, 3>(p, smem, static_cast<int>(blocks), stream);
+        default: return run<A4, 2>(p, smem, static_cast<int>(blocks), stream);
     }
+}
+
+}  // namespace
+
+mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
+                             cudaStream_t stream, float *partial, const L2Prefetch &pf,
+                             bool force) {
+    const DeviceWeight &d = weight_device(w);
+    WideParams p{};
+    p.X = static_cast<const __nv_bfloat16 *>(X);
+    p.Y = static_cast<__nv_bfloat16 *>(Y);
+    p.Yf = partial;
+    p.pf = pf;
+    return launch<false>(p, d, M, partial == nullptr && d.nnz > 0, force, stream);
+}
+
+mq_status launch_decode_wide_a4(const mq_weight *w, const int8_t *codes, const float *xscale,
+                                int M, void *Y, cudaStream_t stream) {
+    const DeviceWeight &d = weight_device(w);
+    WideParams p{};
+    p.codes = codes;
+    p.xscale = xscale;
+    p.Y = static_cast<__nv_bfloat16 *>(Y);
+    return launch<true>(p, d, M, d.nnz > 0, false, stream);
 }
 
 }  // namespace mq

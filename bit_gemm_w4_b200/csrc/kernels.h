@@ -92,15 +92,23 @@ mq_status launch_decode_wide(const mq_weight *w, const void *X, int M, void *Y,
                              cudaStream_t stream, float *partial = nullptr,
                              const L2Prefetch &pf = L2Prefetch(), bool force = false);
 
+// The wide decode kernel's W4A4 form (8 < M <= 16, layers whose 128-row
+// blocks fill the GPU): activation codes with each 8-column chunk's bytes in
+// the packed codes' k order, fp32 scales [M]. MQ_ERR_UNSUPPORTED (no
+// message) when it does not take the call.
+mq_status launch_decode_wide_a4(const mq_weight *w, const int8_t *codes, const float *xscale,
+                                int M, void *Y, cudaStream_t stream);
+
 // Prefill kernel (prefill.cu): any M >= 1; `partial` as for decode.
 mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
                          cudaStream_t stream, float *partial = nullptr);
 
 // W4A4 (w4a4.cu): per-token int4 quantization of bf16 X into int8 codes
-// [M][K] and fp32 scales [M]; then the fused W4A4 product for M <= 16 from
-// those codes (Y bf16 [M][N]).
+// [M][K] (with `permuted`, each 8-column chunk's bytes in the order
+// (0,4,1,5,2,6,3,7), the form the W4A4 kernels read) and fp32 scales [M];
+// then the fused W4A4 product for M <= 16 from permuted codes (Y bf16).
 mq_status launch_quantize(const void *X, int64_t M, int64_t K, void *codes, float *scales,
-                          cudaStream_t stream);
+                          cudaStream_t stream, bool permuted);
 mq_status launch_decode_a4(const mq_weight *w, const int8_t *codes, const float *xscale, int M,
                            void *Y, cudaStream_t stream);
 

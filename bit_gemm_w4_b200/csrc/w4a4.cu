@@ -11,15 +11,16 @@
 //     token), then every code is clamp(rne(fp32(x / s_x)), -8, 7), written as
 //     int8 [M][K].
 //
-//   decode_a4_kernel: the narrow decode kernel's layout (a CTA owns 16*RT rows,
+//   decode_a4_kernel (M <= 8, and up to 16 on layers too small for the wide
+//     kernel's W4A4 form, decode_wide.cu): the narrow decode kernel's layout (a CTA owns 16*RT rows,
 //     its warps split the K groups, codes stream from HBM into registers) with
 //     integer tensor-core MMAs. A thread's 16-byte load of packed codes holds,
 //     per k-step of 32, one word of row g and one of row g+8; masking the low
 //     and the high nibbles gives four bytes each, and (v | 0x80) - z, then
 //     ^ 0x80, per byte turns them into the int8 codes q - z with no carries
 //     between bytes. mma.sync m16n8k32 s8 x s8 -> s32 sums each group exactly;
-//     the group scale is applied in fp32. The activation codes are staged in
-//     shared memory with the bytes of every 8-column chunk permuted as
+//     the group scale is applied in fp32. The quantization kernel writes the
+//     activation codes with the bytes of every 8-column chunk permuted as
 //     (0,4,1,5,2,6,3,7), the order the nibble interleave of the packed codes
 //     puts the weight bytes in, so both operands meet at the same k.
 //     The residual is walked as in the narrow kernel (a team of lanes per
@@ -43,6 +44,7 @@ struct QuantizeArgs {
     int K;
     int8_t *codes;           // [M][K]
     float *scales;           // [M]
+    int permute;             // store each 8-column chunk's codes in the order (0,4,1,5,2,6,3,7)
 };
 
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_constant__ QuantizeArgs qa) {
@@ -85,7 +87,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
             const uint32_t b16 = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
             int q = __float2int_rn(__fdiv_rn(bf16_bits_to_f32(b16), s));
             q = min(7, max(-8, q));
-            out[i >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (i & 3));
+            const int pos = qa.permute ? (((i & 3) << 1) | (i >> 2)) : i;
+            out[pos >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (pos & 3));
         }
         cr[c] = make_uint2(out[0], out[1]);
     }
@@ -143,22 +146,6 @@ struct A4Batch {
     uint4 w[BG][2];
     uint32_t sz[BG][2];
 };
-
-// D = A * B + C, m16n8k32, s8 inputs, s32 accumulate (exact).
-__device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                             uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Four int8 bytes q - z from four nibbles 0..15 held in the low half of each
-// byte of v: (v | 0x80) - z never borrows across bytes; ^ 0x80 restores sign.
-__device__ __forceinline__ uint32_t codes_minus_zero(uint32_t nib4, uint32_t zz4) {
-    return ((nib4 | 0x80808080u) - zz4) ^ 0x80808080u;
-}
 
 // Byte of activation column `rel` (relative to the staged range) inside its
 // permuted 8-column chunk.
@@ -233,15 +220,11 @@ __global__ void __launch_bounds__(A4Cfg<MX, RT, S, BG, CS>::THREADS)
     }
     pdl_wait();  // the codes of X come from the quantization kernel
     {
-        const int k_lo = g_lo * 128, per_row = (g_hi - g_lo) * 16;  // 8-byte chunks
-        for (int m = 0; m < M; ++m) {
-            const uint2 *src = reinterpret_cast<const uint2 *>(p.codes + static_cast<size_t>(m) * K + k_lo);
-            uint2 *dst = reinterpret_cast<uint2 *>(smem + L.x + m * L.xrs);
-            for (int c = threadIdx.x; c < per_row; c += C::THREADS) {
-                const uint2 v = src[c];
-                dst[c] = make_uint2(__byte_perm(v.x, v.y, 0x5140), __byte_perm(v.x, v.y, 0x7362));
-            }
-        }
+        // the codes arrive with each 8-column chunk already permuted
+        const int k_lo = g_lo * 128, per_row = (g_hi - g_lo) * 8;  // 16-byte chunks
+        for (int m = 0; m < M; ++m)
+            for (int c = threadIdx.x; c < per_row; c += C::THREADS)
+                cp_async16(smem + L.x + m * L.xrs + 16 * c, p.codes + static_cast<size_t>(m) * K + k_lo + 16 * c);
     }
     cp_async_wait_all();
     __syncthreads();
@@ -495,16 +478,20 @@ mq_status run_a4_cs(const mq_weight *w, const int8_t *codes, const float *xscale
 }  // namespace
 
 mq_status launch_quantize(const void *X, int64_t M, int64_t K, void *codes, float *scales,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, bool permuted) {
     if (M <= 0) return MQ_OK;
     QuantizeArgs a{static_cast<const __nv_bfloat16 *>(X), static_cast<int>(K),
-                   static_cast<int8_t *>(codes), scales};
+                   static_cast<int8_t *>(codes), scales, permuted ? 1 : 0};
     return launch_pdl(quantize_kernel, a, dim3(static_cast<unsigned>(M)), kQThreads, 0, 1, stream,
                       "activation quantization launch");
 }
 
 mq_status launch_decode_a4(const mq_weight *w, const int8_t *codes, const float *xscale, int M,
                            void *Y, cudaStream_t stream) {
+    if (M > 8) {
+        const mq_status st = launch_decode_wide_a4(w, codes, xscale, M, Y, stream);
+        if (st != MQ_ERR_UNSUPPORTED) return st;
+    }
     if (M == 1) {
         // as for the W4A16 kernel: 4-warp CTAs when the 16-row tiles exceed
         // two 8-warp CTAs per SM

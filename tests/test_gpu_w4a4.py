@@ -96,3 +96,37 @@ def test_w4a4_errors(mq, cuda):
     with pytest.raises(mq.MQError) as e:
         w.linear_w4a4(X[:4], workspace=ws)
     assert e.value.status == mq.INVALID_ARG
+
+
+@pytest.mark.parametrize("M,mode", [(9, "rows"), (16, "rows"), (16, "blocks")])
+def test_w4a4_wide_kernel(mq, cuda, M, mode):
+    # a layer tall enough for the wide kernel's W4A4 form (150 128-row
+    # blocks, K = 384: a last stage holding one group)
+    N, K = 19200, 384
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.01, seed=101)
+    X = synth.activations(M, K, seed=102 + M, channels=2, mult=20.0)
+    if mode == "rows":
+        w = mq.Weight.pack(W, 0.05)
+        d = oracle.decompose(W, 0.05)
+    else:
+        w = mq.Weight.pack(W, block_fraction=0.2)
+        d = oracle.decompose_blocks(W, 0.2)
+    Y = w.linear_w4a4(X.cuda())
+    torch.cuda.synchronize()
+    assert w.device_error() == 0
+    r = oracle_check_w4a4(Y, X, d)
+    assert r["ok"], r
+
+
+def test_w4a4_70b_mlp_sampled_rows(mq, cuda):
+    # the 70B MLP at M = 16 through the wide kernel's W4A4 form
+    N, K = synth.WORKLOADS["70b_mlp"]["shapes"][0]
+    W, X, rho = synth.workload_inputs("70b_mlp")
+    w = mq.Weight.pack(W, rho)
+    Y = w.linear_w4a4(X.cuda())
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([np.arange(0, 24), np.arange(N - 24, N),
+                                     np.random.default_rng(1).choice(N, 48, replace=False)]))
+    d = oracle.decompose(np.ascontiguousarray(W[rows]), rho)
+    r = oracle_check_w4a4(Y[:, torch.from_numpy(rows).cuda()], X, d)
+    assert r["ok"], r
