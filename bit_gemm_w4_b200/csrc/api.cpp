@@ -9,8 +9,9 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
-#include <cstring>
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 #include <new>
 #include <string>
@@ -158,6 +159,10 @@ void build_wide_lists(const HostPacked &hp, std::vector<int32_t> &ptr, std::vect
 
 mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **out) {
     *out = nullptr;
+    // Failure injection for tests: MQ_FAULT_ALLOC=1 makes the first device
+    // allocation fail before any CUDA call is made.
+    if (const char *f = std::getenv("MQ_FAULT_ALLOC"); f && std::strcmp(f, "1") == 0)
+        return fail(MQ_ERR_OUT_OF_MEMORY, "device allocation failed (injected by MQ_FAULT_ALLOC=1)");
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "no usable CUDA device");
@@ -534,6 +539,13 @@ mq_status mq_quantize_activations(const void *X, int64_t M, int64_t K, void *cod
     if (!aligned16(X) || !aligned16(codes) || !aligned16(scales))
         return fail(MQ_ERR_INVALID_ARG, "X, codes and scales must be 16-byte aligned");
     return launch_quantize(X, M, K, codes, scales, reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+mq_status mq_selftest_bounded_wait(int64_t limit_cycles, int32_t *results) {
+    if (!results) return fail(MQ_ERR_INVALID_ARG, "results is NULL");
+    if (limit_cycles <= 0 || limit_cycles > (int64_t(1) << 31))
+        return fail(MQ_ERR_INVALID_ARG, "limit_cycles must be in (0, 2^31]");
+    return selftest_bounded_wait(limit_cycles, results);
 }
 
 int64_t mq_w4a4_workspace_bytes(const mq_weight *w, int64_t M) {

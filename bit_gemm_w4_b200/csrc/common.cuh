@@ -71,11 +71,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 
 // Wait for the phase with the given parity to complete. A tight try_wait
 // loop (the instruction itself suspends the thread for a while) that looks
-// at the clock only every 256 polls; gives up after kWaitCycles or once
-// *abort is set, records `code` in *err and sets *abort so that every later
-// wait of the block returns immediately.
+// at the clock only every 256 polls; gives up after `limit` cycles
+// (kWaitCycles unless a self-test asks for less) or once *abort is set,
+// records `code` in *err (global or shared memory) and sets *abort so that
+// every later wait of the block returns immediately.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err, int code,
-                                          volatile int *abort) {
+                                          volatile int *abort, long long limit = kWaitCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
@@ -83,7 +84,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             atomicCAS(err, 0, code);
             *abort = 1;
             return false;

@@ -112,6 +112,11 @@ mq_status launch_quantize(const void *X, int64_t M, int64_t K, void *codes, floa
 mq_status launch_decode_a4(const mq_weight *w, const int8_t *codes, const float *xscale, int M,
                            void *Y, cudaStream_t stream);
 
+// Self-test of the bounded mbarrier wait (selftest.cu): results[0..3] =
+// {a completed phase was seen, the stuck wait returned true, a later wait
+// returned true, the error word}; expected {1, 0, 0, kErrWaitEmpty}.
+mq_status selftest_bounded_wait(long long limit, int32_t *results);
+
 // Separate residual kernel (residual.cu): Y = bf16(partial + X * R^T).
 mq_status launch_residual_merge(const mq_weight *w, const void *X, int64_t M,
                                 const float *partial, void *Y, cudaStream_t stream);

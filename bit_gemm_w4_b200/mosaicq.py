@@ -66,6 +66,7 @@ def _load():
         "mq_linear_unfused": ([vp, vp, i64, vp, vp, ctypes.c_size_t, vp], st),
         "mq_linear_unfused_noalloc": ([vp, vp, i64, vp, vp], st),
         "mq_quantize_activations": ([vp, i64, i64, vp, vp, vp], st),
+        "mq_selftest_bounded_wait": ([i64, ctypes.POINTER(ctypes.c_int32)], st),
         "mq_w4a4_workspace_bytes": ([vp, i64], i64),
         "mq_linear_w4a4": ([vp, vp, i64, vp, vp, ctypes.c_size_t, vp], st),
         "mq_free": ([vp], None),
@@ -151,6 +152,15 @@ def pack_host(W: np.ndarray, rho: float, group: int = 128, *, block_fraction=Non
     _check(_lib.mq_pack_host(_ptr(W), N, K, ctypes.byref(o), ctypes.byref(hp)), "mq_pack_host")
     del keep
     return arrs
+
+
+def selftest_bounded_wait(limit_cycles: int = 1 << 20) -> list:
+    """Run the bounded-wait self-test on the current device (synchronous):
+    [completed phase seen, stuck wait returned, later wait returned, error
+    code]; [1, 0, 0, 2] when the bounded wait works."""
+    out = (ctypes.c_int32 * 4)()
+    _check(_lib.mq_selftest_bounded_wait(int(limit_cycles), out), "mq_selftest_bounded_wait")
+    return list(out)
 
 
 def quantize_activations(X, *, stream=None):

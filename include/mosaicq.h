@@ -131,6 +131,9 @@ typedef struct {
  * unknown residual_blocks; OUT_OF_MEMORY; CUDA. */
 mq_status mq_pack(const float *W_host, int64_t N, int64_t K,
                   const mq_pack_opts *opts, mq_stream stream, mq_weight **out);
+/* (For tests: with the environment variable MQ_FAULT_ALLOC=1, mq_pack and
+ * mq_pack_decomposed fail with OUT_OF_MEMORY at their first device
+ * allocation, before any CUDA call.) */
 
 /* Y[M][N] = X[M][K] * W_hat^T on `stream`, asynchronously: no host sync, no
  * allocation. X and Y are bf16, row-major, device memory of the packing
@@ -239,6 +242,17 @@ mq_status mq_linear_w4a4(const mq_weight *w, const void *X_dev, int64_t M, void 
 void mq_free(mq_weight *w);
 
 /* --- support for tests and benchmarks (not needed for inference) --- */
+
+/* Failure detection self-test, on the current device, synchronous: runs the
+ * bounded mbarrier wait every pipeline uses on a barrier phase that nobody
+ * completes, with a limit of `limit_cycles` clock cycles (at most 2^31; the
+ * pipelines use 2e9). results[0..3] = {a wait on a completed phase returned
+ * true, the stuck wait returned true, a wait after it returned true, the
+ * error code recorded}; a working wait gives {1, 0, 0, 2}: the stuck wait
+ * gave up, recorded code 2 and made the later wait return at once. The GPU
+ * is never hung: the stuck wait ends after its limit.
+ * Errors: INVALID_ARG for NULL results or a limit outside (0, 2^31]; CUDA. */
+mq_status mq_selftest_bounded_wait(int64_t limit_cycles, int32_t *results);
 
 /* Residual entries a pack with these options produces: N * k_n in row mode,
  * (selected blocks) * 1024 in block mode. */

@@ -345,3 +345,9 @@ def test_longest_k_decode(mq, cuda, M):
     w, Y = _run(mq, W, X, 0.002)
     r = oracle_check(Y, X, oracle.decompose(W, 0.002))
     assert r["ok"], r
+
+
+def test_bounded_wait_gives_up(mq, cuda):
+    # a wait on a barrier phase nobody completes ends after its limit with
+    # its code in the error word, and the wait after it returns at once
+    assert mq.selftest_bounded_wait(1 << 20) == [1, 0, 0, 2]

@@ -62,3 +62,14 @@ def test_nonfinite_and_overflow_rejected(mq):
     with pytest.raises(mq.MQError) as e:
         mq.pack_host(W, 0.01)
     assert "overflow" in str(e.value)
+
+
+def test_injected_allocation_failure(mq, monkeypatch):
+    # MQ_FAULT_ALLOC=1: packing fails with OUT_OF_MEMORY at its first device
+    # allocation, before any CUDA call (so this holds without a GPU too)
+    W = np.random.default_rng(0).standard_normal((32, 256)).astype(np.float32) * 0.02
+    monkeypatch.setenv("MQ_FAULT_ALLOC", "1")
+    with pytest.raises(mq.MQError) as e:
+        mq.Weight.pack(W, 0.02, stream=0)      # the default stream: no torch CUDA call
+    assert e.value.status == mq.OUT_OF_MEMORY
+    assert b"MQ_FAULT_ALLOC" in mq.lib().mq_last_error()
