@@ -351,3 +351,30 @@ def test_bounded_wait_gives_up(mq, cuda):
     # a wait on a barrier phase nobody completes ends after its limit with
     # its code in the error word, and the wait after it returns at once
     assert mq.selftest_bounded_wait(1 << 20) == [1, 0, 0, 2]
+
+
+@pytest.mark.parametrize("N,K,M,path", [
+    (200, 384, 1, "auto"),        # narrow decode, ragged tile
+    (200, 384, 13, "auto"),       # narrow decode, 16-token layout
+    (19000, 384, 16, "auto"),     # wide decode kernel
+    (200, 384, 77, "prefill"),    # prefill, ragged tiles
+    (200, 384, 5, "w4a4"),        # W4A4
+    (19000, 384, 12, "w4a4"),     # W4A4 through the wide kernel
+])
+def test_outputs_stay_inside_y(mq, cuda, N, K, M, path):
+    # Y lives inside a canary-filled buffer; only its M x N elements may change
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.01, seed=107)
+    w = mq.Weight.pack(W, 0.05)
+    X = synth.activations(M, K, seed=108).cuda()
+    pad = 4096
+    canary = torch.full((pad + M * N + pad,), -7.5, dtype=torch.bfloat16, device="cuda")
+    Y = canary[pad:pad + M * N].view(M, N)
+    if path == "w4a4":
+        w.linear_w4a4(X, Y)
+    else:
+        w.linear(X, Y, path=path)
+    torch.cuda.synchronize()
+    assert torch.all(canary[:pad] == -7.5) and torch.all(canary[pad + M * N:] == -7.5)
+    fresh = w.linear_w4a4(X) if path == "w4a4" else w.linear(X, path=path)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, fresh)
