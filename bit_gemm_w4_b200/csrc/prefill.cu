@@ -401,8 +401,6 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
         const int n = 32 * q + lane;   // weight row within the tile (= lane)
         const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16) + T_A;
         int it = 0, pc = 0;
-        // the residual groups this warp wrote in the last NSLOT stages (oldest last)
-        int h0[NSLOT] = {0, 0, 0, 0}, h1[NSLOT] = {0, 0, 0, 0};
         bool ok = true;
         for (int t = t_begin; ok && t < t_end; ++t) {
             const int row = (t / p.m_tiles) * BN + n;
@@ -413,9 +411,11 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                 const int a = it & (NSLOT - 1), ps = pc & (NPSLOT - 1);
                 const uint32_t szw = valid ? __ldg(szrow + (i >> 1)) : 0u;
                 int g0 = 0, g1 = 0;  // this warp's residual group of the stage
+                uint32_t v0 = 0u;    // its first entry per lane, requested before the waits
                 if (res) {
                     g0 = __ldg(gptr + 4 * i);
                     g1 = __ldg(gptr + 4 * i + 1);
+                    if (g0 + lane < g1) v0 = __ldg(p.stage_ent + g0 + lane);
                 }
                 if ((pi == 0 &&
                      !mbar_wait_warp(&pfull[ps], (pc >> 1) & 1, p.err, kErrWaitFull, abort_flag)) ||
@@ -452,26 +452,19 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                 bool has = false;
                 if (res) {
                     uint8_t *rt = smem + L.rtile + a * R_BYTES;
-                    // clear this warp's entries of the stage that used the slot
-                    // NSLOT stages ago, then write the stage's entries; an entry
-                    // word holds row, column and the bf16 code ready to store
-                    const int o0 = h0[NSLOT - 1], o1 = h1[NSLOT - 1];
+                    // zero this warp's 32 rows of the slot (the stage that used it
+                    // NSLOT stages ago may have left entries there), then write the
+                    // stage's entries; an entry word holds row, column and the bf16
+                    // code ready to store
+                    if (it >= NSLOT) {
+                        uint8_t *rq = rt + 32 * q * 128;
 #pragma unroll
-                    for (int h = NSLOT - 1; h > 0; --h) {
-                        h0[h] = h0[h - 1];
-                        h1[h] = h1[h - 1];
+                        for (int k = 0; k < 8; ++k)
+                            sts128(rq + 512 * k + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
                     }
-                    h0[0] = g0;
-                    h1[0] = g1;
-                    if (it >= NSLOT)
-                        for (int e = o0 + lane; e < o1; e += 32) {
-                            const uint32_t v = __ldg(p.stage_ent + e);
-                            const int r = v & 127, c = (v >> 8) & 63;
-                            sts16(rt + r * 128 + (((c >> 3) ^ (r & 7)) << 4) + (c & 7) * 2, 0);
-                        }
                     __syncwarp();
                     for (int e = g0 + lane; e < g1; e += 32) {
-                        const uint32_t v = __ldg(p.stage_ent + e);
+                        const uint32_t v = (e == g0 + lane) ? v0 : __ldg(p.stage_ent + e);
                         const int r = v & 127, c = (v >> 8) & 63;
                         sts16(rt + r * 128 + (((c >> 3) ^ (r & 7)) << 4) + (c & 7) * 2,
                               static_cast<uint16_t>(v >> 16));
