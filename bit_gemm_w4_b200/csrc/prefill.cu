@@ -407,15 +407,34 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
             const bool valid = row < p.N;
             const uint32_t *szrow = p.sz + static_cast<size_t>(row) * Gp;
             const int32_t *gptr = res ? p.stage_ptr + (static_cast<size_t>(t / p.m_tiles) * nk) * 4 + q : nullptr;
+            // The residual entries are requested ahead of use: a stage's group
+            // bounds two stages early, its first entry per lane one stage early,
+            // so neither global load sits on the path from the waits to the MMA.
+            int na0 = 0, na1 = 0, nb0 = 0, nb1 = 0;
+            uint32_t nv = 0u;
+            if (res) {
+                na0 = __ldg(gptr);
+                na1 = __ldg(gptr + 1);
+                if (na0 + lane < na1) nv = __ldg(p.stage_ent + na0 + lane);
+                if (nk > 1) {
+                    nb0 = __ldg(gptr + 4);
+                    nb1 = __ldg(gptr + 5);
+                }
+            }
             for (int i = 0, pi = 0; i < nk; ++i, ++it) {
                 const int a = it & (NSLOT - 1), ps = pc & (NPSLOT - 1);
                 const uint32_t szw = valid ? __ldg(szrow + (i >> 1)) : 0u;
-                int g0 = 0, g1 = 0;  // this warp's residual group of the stage
-                uint32_t v0 = 0u;    // its first entry per lane, requested before the waits
+                // this warp's residual group of the stage and its first entry per lane
+                const int g0 = na0, g1 = na1;
+                const uint32_t v0 = nv;
                 if (res) {
-                    g0 = __ldg(gptr + 4 * i);
-                    g1 = __ldg(gptr + 4 * i + 1);
-                    if (g0 + lane < g1) v0 = __ldg(p.stage_ent + g0 + lane);
+                    na0 = nb0;
+                    na1 = nb1;
+                    nv = (i + 1 < nk && na0 + lane < na1) ? __ldg(p.stage_ent + na0 + lane) : 0u;
+                    if (i + 2 < nk) {
+                        nb0 = __ldg(gptr + 4 * (i + 2));
+                        nb1 = __ldg(gptr + 4 * (i + 2) + 1);
+                    }
                 }
                 if ((pi == 0 &&
                      !mbar_wait_warp(&pfull[ps], (pc >> 1) & 1, p.err, kErrWaitFull, abort_flag)) ||
