@@ -66,10 +66,11 @@ constexpr int T_BYTES = X_BYTES;      // one TMA stage
 constexpr int PSLOT_BYTES = BN * 32 * 4;  // packed codes of up to four stages
 constexpr int NPSLOT = 2;
 constexpr int R_BYTES = BN * BK * 2;  // one residual code tile
-constexpr int NSLOT = 4;              // operand slots (dense in TMEM, residual in smem)
+constexpr int NSLOT = 4;   // operand slots with the residual (dense in TMEM, residual in smem)
+constexpr int MAX_NS = 8;  // operand slots without it (R's columns hold four more)
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t T_D = 0, T_R = 256, T_A = 384;  // column bases
-constexpr uint32_t A_SLOT = 32;                    // columns per operand slot
+constexpr uint32_t T_D = 0, T_R = 256;  // column bases; the operand slots end the columns
+constexpr uint32_t A_SLOT = 32;         // columns per operand slot
 static_assert(T_BYTES % 1024 == 0 && R_BYTES % 1024 == 0, "1024-byte swizzle alignment");
 static_assert(2 * T_BYTES >= BM * BN * 2, "the output tile is staged in the TMA ring");
 
@@ -98,8 +99,8 @@ struct SmemLayout {
         pring = XS * CX * T_BYTES;  // the X ring starts at 0
         rtile = pring + NPSLOT * PSLOT_BYTES;
         rflag = rtile + (residual ? NSLOT * R_BYTES : 0);
-        bars = rflag + NSLOT * 4 * 4;
-        tmem_slot = bars + (2 * MAX_XS + 2 * NSLOT + 2 * NPSLOT + 8) * 8;
+        bars = rflag + MAX_NS * 4 * 4;
+        tmem_slot = bars + (2 * MAX_XS + MAX_NS + 2 * NPSLOT + 8) * 8;
         abort = tmem_slot + 16;
         total = abort + 16;
     }
@@ -205,11 +206,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// NS operand slots, handed over in pairs: 4 when the residual is fused (its
+// accumulator takes tensor-memory columns 256..383), else 8.
+template <int NS>
 __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
+    static_assert(NS == NSLOT || NS == MAX_NS, "operand slot count");
+    constexpr int NP = NS / 2;                         // slot pairs
+    constexpr int NS_LOG = NS == 8 ? 3 : 2;
+    constexpr uint32_t T_A = TMEM_COLS - NS * A_SLOT;  // first operand slot column
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const bool res = p.with_residual != 0;
+    const bool res = NS == NSLOT && p.with_residual != 0;
     const SmemLayout L(p.XS, p.CX, res);
     const int XS = p.XS, CX = p.CX;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -219,20 +227,20 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
     const int t_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * p.tiles / gridDim.x);
     const int t_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * p.tiles / gridDim.x);
 
-    volatile uint32_t *rflag = reinterpret_cast<volatile uint32_t *>(smem + L.rflag);  // [NSLOT][4]
+    volatile uint32_t *rflag = reinterpret_cast<volatile uint32_t *>(smem + L.rflag);  // [NS][4]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *full = bars;                 // [XS] X copy landed
     uint64_t *empty = bars + MAX_XS;       // [XS] MMAs reading the X copy done
     // operand slots go back and forth in pairs (one 128-column group)
-    uint64_t *bready = bars + 2 * MAX_XS;  // [2] operand slot pair written
-    uint64_t *bempty = bready + NSLOT;     // [2] MMAs reading the slot pair done
-    uint64_t *dfull = bempty + NSLOT;      // [2] group partial ready in TMEM
+    uint64_t *bready = bars + 2 * MAX_XS;   // [NP] operand slot pair written
+    uint64_t *bempty = bready + MAX_NS / 2;  // [NP] MMAs reading the slot pair done
+    uint64_t *dfull = bempty + MAX_NS / 2;   // [2] group partial ready in TMEM
     uint64_t *dempty = dfull + 2;          // [2] epilogue done with the TMEM buffer
     uint64_t *rfull = dempty + 2;          // every MMA of the tile complete
     uint64_t *rempty = rfull + 1;          // epilogue done with the tile's R
     uint64_t *pfull = rempty + 1;          // [NPSLOT] packed codes landed
     uint64_t *pempty = pfull + NPSLOT;     // [NPSLOT] dequant done with the packed codes
-    static_assert(NSLOT == 4 && NPSLOT == 2, "slot arithmetic below uses shifts");
+    static_assert(NPSLOT == 2, "slot arithmetic below uses shifts");
     const int spl = p.pw / 8;              // stages per packed-code load
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.tmem_slot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.abort);
@@ -242,7 +250,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NP; ++b) {
             mbar_init(&bready[b], 4);
             mbar_init(&bempty[b], 1);
         }
@@ -336,21 +344,21 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
             for (int t = t_begin, j = 0; ok && t < t_end; ++t, ++j, gg0 += G) {
                 // two stages (one group, one operand slot pair) per step
                 for (int i = 0, xi = 0; i < nk; i += 2, it += 2) {
-                    const int gg = gg0 + (i >> 1), b = gg & 1, pp = (it >> 1) & 1;
+                    const int gg = gg0 + (i >> 1), b = gg & 1, pp = (it >> 1) & (NP - 1);
                     if (gg >= 2 &&
                         !mbar_wait(&dempty[b], ((gg >> 1) - 1) & 1, p.err, kErrWaitMma, abort_flag)) {
                         ok = false;
                         break;
                     }
                     if ((xi == 0 && !mbar_wait(&full[xs], xround & 1, p.err, kErrWaitFull, abort_flag)) ||
-                        !mbar_wait(&bready[pp], (it >> 2) & 1, p.err, kErrWaitFull, abort_flag)) {
+                        !mbar_wait(&bready[pp], (it >> NS_LOG) & 1, p.err, kErrWaitFull, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const int a = (it + h) & (NSLOT - 1);
+                        const int a = (it + h) & (NS - 1);
                         const uint64_t xd = sw128_desc(smem_u32(smem + (xs * CX + xi + h) * T_BYTES));
                         const uint32_t at = tmem + T_A + a * A_SLOT;
 #pragma unroll
@@ -421,9 +429,15 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     nb1 = __ldg(gptr + 5);
                 }
             }
+            // the scale / zero word of the next group is requested a group early,
+            // so its latency is not exposed behind waits that complete at once
+            uint32_t sz_next = valid ? __ldg(szrow) : 0u, szw = 0u;
             for (int i = 0, pi = 0; i < nk; ++i, ++it) {
-                const int a = it & (NSLOT - 1), ps = pc & (NPSLOT - 1);
-                const uint32_t szw = valid ? __ldg(szrow + (i >> 1)) : 0u;
+                const int a = it & (NS - 1), ps = pc & (NPSLOT - 1);
+                if ((i & 1) == 0) {
+                    szw = sz_next;
+                    sz_next = (valid && (i >> 1) + 1 < G) ? __ldg(szrow + (i >> 1) + 1) : 0u;
+                }
                 // this warp's residual group of the stage and its first entry per lane
                 const int g0 = na0, g1 = na1;
                 const uint32_t v0 = nv;
@@ -438,9 +452,9 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                 }
                 if ((pi == 0 &&
                      !mbar_wait_warp(&pfull[ps], (pc >> 1) & 1, p.err, kErrWaitFull, abort_flag)) ||
-                    ((it & 1) == 0 && it >= NSLOT &&
-                     !mbar_wait_warp(&bempty[(it >> 1) & 1], ((it >> 2) - 1) & 1, p.err, kErrWaitMma,
-                                     abort_flag))) {
+                    ((it & 1) == 0 && it >= NS &&
+                     !mbar_wait_warp(&bempty[(it >> 1) & (NP - 1)], ((it >> NS_LOG) - 1) & 1, p.err,
+                                     kErrWaitMma, abort_flag))) {
                     ok = false;
                     break;
                 }
@@ -497,7 +511,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     tmem_st_wait();  // both stages' codes are in tensor memory
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bready[(it >> 1) & 1]);
+                    if (lane == 0) mbar_arrive(&bready[(it >> 1) & (NP - 1)]);
                 }
             }
         }
@@ -626,7 +640,9 @@ mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
     if (dev < 0 || dev >= 64) return fail(MQ_ERR_UNSUPPORTED, "device ordinal above 63");
     if (!configured[dev]) {
-        if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(prefill_kernel<NSLOT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 227 * 1024) != cudaSuccess ||
+            cudaFuncSetAttribute(prefill_kernel<MAX_NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  227 * 1024) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             sms[dev] <= 0)
@@ -635,7 +651,10 @@ mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
     }
     // one CTA per SM (its shared memory and 512 TMEM columns allow no second)
     const int grid = static_cast<int>(std::min<int64_t>(tiles, sms[dev]));
-    prefill_kernel<<<grid, THREADS, smem, stream>>>(p);
+    if (p.with_residual)
+        prefill_kernel<NSLOT><<<grid, THREADS, smem, stream>>>(p);
+    else
+        prefill_kernel<MAX_NS><<<grid, THREADS, smem, stream>>>(p);
     cudaError_t e = cudaPeekAtLastError();
     if (e != cudaSuccess)
         return fail(MQ_ERR_CUDA, std::string("prefill launch: ") + cudaGetErrorString(e));
