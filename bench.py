@@ -568,6 +568,7 @@ PROFILE_CASES = {
     "decode-28672x8192-m16": (28672, 8192, 16, 0.01, "auto"),
     "prefill-14336x4096-m256": (14336, 4096, 256, 0.005, "prefill"),
     "prefill-14336x4096-m2048": (14336, 4096, 2048, 0.005, "prefill"),
+    "prefill-14336x4096-m2048-dense": (14336, 4096, 2048, 0.0, "prefill"),
 }
 
 
