@@ -305,6 +305,22 @@ bool encode_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K, int chu
     return r == CUDA_SUCCESS;
 }
 
+bool encode_codes_map(CUtensorMap *map, const void *codes, int64_t M, int64_t K, int chunks) {
+    // int8 activation codes [M][K] viewed as [K/128][M][128]: one box is
+    // `chunks` consecutive 128-column tiles [128 rows][128 bytes], each
+    // 128-byte swizzled (the same 16 KB tile as 64 bf16 columns)
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(K / 128)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), 128};
+    cuuint32_t box[3] = {128, 128, static_cast<cuuint32_t>(chunks)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(codes), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace mq
 
 using namespace mq;
@@ -558,7 +574,6 @@ mq_status mq_linear_w4a4(const mq_weight *w, const void *X, int64_t M, void *Y, 
     if (!w) return fail(MQ_ERR_INVALID_ARG, "weight handle is NULL");
     if (M < 0) return fail(MQ_ERR_INVALID_ARG, "M must be >= 0");
     if (M == 0) return MQ_OK;
-    if (M > 16) return fail(MQ_ERR_UNSUPPORTED, "W4A4 serves M <= 16 (the decode regime)");
     if (!X || !Y || !workspace) return fail(MQ_ERR_INVALID_ARG, "X, Y or workspace is NULL");
     if (!aligned16(X) || !aligned16(Y) || !aligned16(workspace))
         return fail(MQ_ERR_INVALID_ARG, "X, Y and workspace must be 16-byte aligned");
@@ -572,9 +587,12 @@ mq_status mq_linear_w4a4(const mq_weight *w, const void *X, int64_t M, void *Y, 
     int8_t *codes = static_cast<int8_t *>(workspace);
     float *scales = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
                                               (M * w->d.K + 15) / 16 * 16);
+    if (M > (int64_t(1) << 23)) return fail(MQ_ERR_UNSUPPORTED, "W4A4: M above 2^23");
     mq_status st = launch_quantize(X, M, w->d.K, codes, scales, s, true);
     if (st) return st;
-    return launch_decode_a4(w, codes, scales, static_cast<int>(M), Y, s);
+    // M <= 16: the narrow and wide decode kernels; above, the tcgen05 prefill kernel
+    if (M <= 16) return launch_decode_a4(w, codes, scales, static_cast<int>(M), Y, s);
+    return launch_prefill_a4(w, codes, scales, M, Y, s);
 }
 
 }  // extern "C"

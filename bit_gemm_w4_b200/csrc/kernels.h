@@ -62,6 +62,9 @@ const PrefillMaps *prefill_maps(const mq_weight *w);
 // bf16 X [M][K] row-major as a 3D view [K/64][M][64]; one box holds `chunks`
 // consecutive [128 rows][64 columns] tiles, each 128-byte swizzled.
 bool encode_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K, int chunks);
+// int8 activation codes [M][K] (K a multiple of 128) as the prefill kernel's
+// W4A4 X operand: boxes of `chunks` 128-column tiles [128][128 bytes].
+bool encode_codes_map(CUtensorMap *map, const void *codes, int64_t M, int64_t K, int chunks);
 const DeviceWeight &weight_device(const mq_weight *w);
 
 // Streaming multiprocessors of the current device (cached per device).
@@ -102,6 +105,11 @@ mq_status launch_decode_wide_a4(const mq_weight *w, const int8_t *codes, const f
 // Prefill kernel (prefill.cu): any M >= 1; `partial` as for decode.
 mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
                          cudaStream_t stream, float *partial = nullptr);
+
+// The prefill kernel's W4A4 form (K a multiple of 256): permuted int8
+// activation codes [M][K] and fp32 scales [M]; int8 tensor-core MMAs.
+mq_status launch_prefill_a4(const mq_weight *w, const int8_t *codes, const float *xscale, int64_t M,
+                            void *Y, cudaStream_t stream);
 
 // W4A4 (w4a4.cu): per-token int4 quantization of bf16 X into int8 codes
 // [M][K] (with `permuted`, each 8-column chunk's bytes in the order

@@ -75,12 +75,13 @@ static_assert(T_BYTES % 1024 == 0 && R_BYTES % 1024 == 0, "1024-byte swizzle ali
 static_assert(2 * T_BYTES >= BM * BN * 2, "the output tile is staged in the TMA ring");
 
 struct PrefillParams {
-    CUtensorMap tm_x;  // X [M][K] bf16, box [128][64], 128B swizzle
+    CUtensorMap tm_x;  // X [M][K] bf16 (box [128][64]) or int8 codes (box [128][128]), 128B swizzle
     CUtensorMap tm_w;  // qweight [N][K/8] u32, box [128][8]
     const int32_t *stage_ptr;   // residual groups per (tile, stage, quadrant)
     const uint32_t *stage_ent;
     const uint16_t *rscale;
     const uint32_t *sz;  // [N][Gp] scale | zero << 16
+    const float *xscale;  // [M] per-token activation scales (W4A4), else NULL
     __nv_bfloat16 *Y;
     float *Yf;
     int *err;
@@ -136,18 +137,30 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
            (static_cast<uint64_t>(2) << 61);
 }
 
-// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128, N = 128.
+// Instruction descriptors, both operands K-major, M = 128, N = 128:
+// bf16 x bf16 -> fp32 (kind::f16), and s8 x s8 -> s32 (kind::i8, W4A4).
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
                             (static_cast<uint32_t>(BM >> 4) << 24);
+constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) |
+                              (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
 
-// D[tmem] (+)= A[smem] * B[smem]^T, both K-major shared-memory tiles.
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major shared-memory tiles; A4
+// selects the int8 kind (32 k per step) over bf16 (16 k per step).
+template <bool A4>
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
-        : "memory");
+    if constexpr (A4)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(kIdescI8), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+            : "memory");
 }
 
 __device__ __forceinline__ void sts16(void *p, uint16_t v) {
@@ -156,13 +169,27 @@ __device__ __forceinline__ void sts16(void *p, uint16_t v) {
 
 // D[tmem] (+)= A[tmem] * B[smem]^T: A is M x 16 bf16 in tensor memory (lane =
 // row, two codes per 32-bit column), B an N x 16 K-major shared-memory tile.
+template <bool A4>
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
                                        uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
-        : "memory");
+    if constexpr (A4)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "r"(a_tmem), "l"(bdesc), "r"(kIdescI8), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "r"(a_tmem), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+            : "memory");
+}
+
+// An int32 of magnitude below 2^22 as fp32, exactly, with two adds: placed in
+// the mantissa of 1.5 * 2^23 (ulp 1) and the bias taken off again.
+__device__ __forceinline__ float small_int_to_f32(uint32_t bits) {
+    return __int_as_float(static_cast<int>(bits) + 0x4B400000) - 12582912.0f;
 }
 
 // 32 lanes x 32 columns of 32-bit values: thread i writes lane (base + i).
@@ -208,9 +235,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 // NS operand slots, handed over in pairs: 4 when the residual is fused (its
 // accumulator takes tensor-memory columns 256..383), else 8.
-template <int NS>
+// A4: the W4A4 form. X is int8 activation codes (each 8-column chunk in the
+// packed codes' k order), a stage is 128 columns (one quantization group, the
+// same 16 KB X tile and 32 tensor-memory columns as 64 bf16 columns), the
+// dequant warps write int8 codes q - z, the MMAs are kind::i8 into int32, and
+// the epilogue scales by s[n][g], s_r[n] and the token's s_x.
+template <int NS, bool A4>
 __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
     static_assert(NS == NSLOT || NS == MAX_NS, "operand slot count");
+    constexpr int SK = A4 ? 128 : BK;  // K columns per stage
+    constexpr int WPS = SK / 8;        // packed words per row and stage
     constexpr int NP = NS / 2;                         // slot pairs
     constexpr int NS_LOG = NS == 8 ? 3 : 2;
     constexpr uint32_t T_A = TMEM_COLS - NS * A_SLOT;  // first operand slot column
@@ -221,7 +255,8 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
     const SmemLayout L(p.XS, p.CX, res);
     const int XS = p.XS, CX = p.CX;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nk = p.K / BK;
+    const int nk = p.K / SK;     // stages per tile (even: K is a multiple of 256 for A4)
+    const int nls = p.K / BK;    // residual list stages per tile (64 columns each)
     const int G = p.G, Gp = p.Gp;
     // this CTA's tiles
     const int t_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * p.tiles / gridDim.x);
@@ -241,7 +276,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
     uint64_t *pfull = rempty + 1;          // [NPSLOT] packed codes landed
     uint64_t *pempty = pfull + NPSLOT;     // [NPSLOT] dequant done with the packed codes
     static_assert(NPSLOT == 2, "slot arithmetic below uses shifts");
-    const int spl = p.pw / 8;              // stages per packed-code load
+    const int spl = p.pw / WPS;            // stages per packed-code load
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.tmem_slot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.abort);
 
@@ -300,7 +335,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                             break;
                         }
                         mbar_arrive_expect_tx(&pfull[ps], BN * p.pw * 4);
-                        tma_load_2d(smem + L.pring + ps * PSLOT_BYTES, &p.tm_w, &pfull[ps], i * (BK / 8), n0);
+                        tma_load_2d(smem + L.pring + ps * PSLOT_BYTES, &p.tm_w, &pfull[ps], i * WPS, n0);
                         ++pc;
                     }
                     if (++pi == spl) pi = 0;
@@ -342,10 +377,11 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
             int xs = 0, xround = 0;  // X slot being read, times the ring wrapped
             bool ok = true;
             for (int t = t_begin, j = 0; ok && t < t_end; ++t, ++j, gg0 += G) {
-                // two stages (one group, one operand slot pair) per step
+                // two stages (one operand slot pair; one group, or two for A4) per step
                 for (int i = 0, xi = 0; i < nk; i += 2, it += 2) {
-                    const int gg = gg0 + (i >> 1), b = gg & 1, pp = (it >> 1) & (NP - 1);
-                    if (gg >= 2 &&
+                    const int pp = (it >> 1) & (NP - 1);
+                    int gg = gg0 + (i >> 1), b = gg & 1;
+                    if (!A4 && gg >= 2 &&
                         !mbar_wait(&dempty[b], ((gg >> 1) - 1) & 1, p.err, kErrWaitMma, abort_flag)) {
                         ok = false;
                         break;
@@ -358,12 +394,23 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     tc_fence_after();
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
+                        if constexpr (A4) {  // each stage is a group of its own
+                            gg = gg0 + i + h;
+                            b = gg & 1;
+                            if (gg >= 2 && !mbar_wait(&dempty[b], ((gg >> 1) - 1) & 1, p.err,
+                                                      kErrWaitMma, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                        }
                         const int a = (it + h) & (NS - 1);
                         const uint64_t xd = sw128_desc(smem_u32(smem + (xs * CX + xi + h) * T_BYTES));
                         const uint32_t at = tmem + T_A + a * A_SLOT;
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            mma_ts(tmem + T_D + b * BM, at + 8 * kk, xd + 2 * kk, (h | kk) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ts<A4>(tmem + T_D + b * BM, at + 8 * kk, xd + 2 * kk,
+                                       ((A4 ? 0 : h) | kk) ? 1u : 0u);
                         // stage 0 always runs, so R is initialized; it may be
                         // overwritten once the epilogue has read the previous tile's R
                         if (res && (rflag[4 * a] | rflag[4 * a + 1] | rflag[4 * a + 2] | rflag[4 * a + 3])) {
@@ -376,9 +423,10 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                             }
                             const uint64_t rd = sw128_desc(smem_u32(smem + L.rtile + a * R_BYTES));
 #pragma unroll
-                            for (int kk = 0; kk < BK / 16; ++kk)
-                                mma_ss(tmem + T_R, rd + 2 * kk, xd + 2 * kk, ((i + h) | kk) ? 1u : 0u);
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_ss<A4>(tmem + T_R, rd + 2 * kk, xd + 2 * kk, ((i + h) | kk) ? 1u : 0u);
                         }
+                        if constexpr (A4) mma_commit(&dfull[b]);
                     }
                     if (!ok) break;
                     xi += 2;
@@ -391,7 +439,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                         }
                     }
                     mma_commit(&bempty[pp]);
-                    mma_commit(&dfull[b]);
+                    if constexpr (!A4) mma_commit(&dfull[b]);
                 }
                 // the epilogue waits for each tile's completion with the tile's parity,
                 // so it must have taken the previous one first
@@ -414,13 +462,13 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
             const int row = (t / p.m_tiles) * BN + n;
             const bool valid = row < p.N;
             const uint32_t *szrow = p.sz + static_cast<size_t>(row) * Gp;
-            const int32_t *gptr = res ? p.stage_ptr + (static_cast<size_t>(t / p.m_tiles) * nk) * 4 + q : nullptr;
+            const int32_t *gptr = res ? p.stage_ptr + (static_cast<size_t>(t / p.m_tiles) * nls) * 4 + q : nullptr;
             // The residual entries are requested ahead of use: a stage's group
             // bounds two stages early, its first entry per lane one stage early,
             // so neither global load sits on the path from the waits to the MMA.
             int na0 = 0, na1 = 0, nb0 = 0, nb1 = 0;
             uint32_t nv = 0u;
-            if (res) {
+            if (!A4 && res) {
                 na0 = __ldg(gptr);
                 na1 = __ldg(gptr + 1);
                 if (na0 + lane < na1) nv = __ldg(p.stage_ent + na0 + lane);
@@ -432,16 +480,17 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
             // the scale / zero word of the next group is requested a group early,
             // so its latency is not exposed behind waits that complete at once
             uint32_t sz_next = valid ? __ldg(szrow) : 0u, szw = 0u;
+            constexpr int SPG = A4 ? 1 : 2;  // stages per quantization group
             for (int i = 0, pi = 0; i < nk; ++i, ++it) {
                 const int a = it & (NS - 1), ps = pc & (NPSLOT - 1);
-                if ((i & 1) == 0) {
+                if (i % SPG == 0) {
                     szw = sz_next;
-                    sz_next = (valid && (i >> 1) + 1 < G) ? __ldg(szrow + (i >> 1) + 1) : 0u;
+                    sz_next = (valid && i / SPG + 1 < G) ? __ldg(szrow + i / SPG + 1) : 0u;
                 }
                 // this warp's residual group of the stage and its first entry per lane
                 const int g0 = na0, g1 = na1;
                 const uint32_t v0 = nv;
-                if (res) {
+                if (!A4 && res) {
                     na0 = nb0;
                     na1 = nb1;
                     nv = (i + 1 < nk && na0 + lane < na1) ? __ldg(p.stage_ent + na0 + lane) : 0u;
@@ -460,26 +509,45 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                 }
                 tc_fence_after();
                 const uint32_t z = static_cast<uint32_t>(half_bits_to_f32(szw >> 16));
-                const uint32_t zz = (0x4300u | z) * 0x00010001u;  // bf16x2 (128 + z)
-                // this stage's two 16-byte chunks of the row (128-byte swizzle when pw = 32)
+                // this stage's 16-byte chunks of the row (128-byte swizzle when pw = 32):
+                // two for 64 bf16 columns, four for 128 int8 columns
                 const uint8_t *prow = smem + L.pring + ps * PSLOT_BYTES + n * (p.pw * 4);
-                const int c0 = 2 * pi, sw = (p.pw == 32) ? (n & 7) : 0;
-                const uint4 w0 = lds128(prow + ((c0 ^ sw) << 4));
-                const uint4 w1 = lds128(prow + (((c0 + 1) ^ sw) << 4));
+                const int c0 = (WPS / 4) * pi, sw = (p.pw == 32) ? (n & 7) : 0;
+                uint32_t words[WPS];
+#pragma unroll
+                for (int u = 0; u < WPS / 4; ++u) {
+                    const uint4 wv = lds128(prow + (((c0 + u) ^ sw) << 4));
+                    words[4 * u] = wv.x;
+                    words[4 * u + 1] = wv.y;
+                    words[4 * u + 2] = wv.z;
+                    words[4 * u + 3] = wv.w;
+                }
                 if (++pi == spl || i == nk - 1) {
                     pi = 0;
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pempty[ps]);
                     ++pc;
                 }
-                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
                 uint32_t codes[32];
+                if constexpr (A4) {
+                    // a word's low nibbles are its columns in positions 0-3 of the
+                    // chunk's code order, the high nibbles positions 4-7: one
+                    // tensor-memory column of four int8 codes q - z each
+                    const uint32_t zz = z * 0x01010101u;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    // pair j of word c holds columns (8c + 2j, 8c + 2j + 1)
+                    for (int c = 0; c < 16; ++c) {
+                        codes[2 * c] = codes_minus_zero(words[c] & 0x0F0F0F0Fu, zz);
+                        codes[2 * c + 1] = codes_minus_zero((words[c] >> 4) & 0x0F0F0F0Fu, zz);
+                    }
+                } else {
+                    const uint32_t zz = (0x4300u | z) * 0x00010001u;  // bf16x2 (128 + z)
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        codes[4 * c + jj] = bf16x2_sub(nib_pair_bias128(words[c] >> (4 * jj)), zz);
+                    for (int c = 0; c < 8; ++c) {
+                        // pair j of word c holds columns (8c + 2j, 8c + 2j + 1)
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj)
+                            codes[4 * c + jj] = bf16x2_sub(nib_pair_bias128(words[c] >> (4 * jj)), zz);
+                    }
                 }
                 tmem_st32(tl + a * A_SLOT, codes);
                 bool has = false;
@@ -496,14 +564,35 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                             sts128(rq + 512 * k + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
                     }
                     __syncwarp();
-                    for (int e = g0 + lane; e < g1; e += 32) {
-                        const uint32_t v = (e == g0 + lane) ? v0 : __ldg(p.stage_ent + e);
-                        const int r = v & 127, c = (v >> 8) & 63;
-                        sts16(rt + r * 128 + (((c >> 3) ^ (r & 7)) << 4) + (c & 7) * 2,
-                              static_cast<uint16_t>(v >> 16));
+                    if constexpr (A4) {
+                        // the two 64-column list stages of this 128-column stage; an
+                        // int8 code goes to its column's position in the chunk's order
+                        int cnt = 0;
+#pragma unroll
+                        for (int sub = 0; sub < 2; ++sub) {
+                            const int e0 = __ldg(gptr + 4 * (2 * i + sub));
+                            const int e1 = __ldg(gptr + 4 * (2 * i + sub) + 1);
+                            cnt += e1 - e0;
+                            for (int e = e0 + lane; e < e1; e += 32) {
+                                const uint32_t v = __ldg(p.stage_ent + e);
+                                const int r = v & 127, c = ((v >> 8) & 63) + 64 * sub;
+                                const int cp = (c & ~7) | ((c & 3) << 1) | ((c >> 2) & 1);
+                                const int q8 = static_cast<int>(bf16_bits_to_f32(v >> 16));
+                                sts_u8(rt + r * 128 + (((cp >> 4) ^ (r & 7)) << 4) + (cp & 15),
+                                       static_cast<uint8_t>(q8 & 0xFF));
+                            }
+                        }
+                        has = cnt > 0 || i == 0;
+                    } else {
+                        for (int e = g0 + lane; e < g1; e += 32) {
+                            const uint32_t v = (e == g0 + lane) ? v0 : __ldg(p.stage_ent + e);
+                            const int r = v & 127, c = (v >> 8) & 63;
+                            sts16(rt + r * 128 + (((c >> 3) ^ (r & 7)) << 4) + (c & 7) * 2,
+                                  static_cast<uint16_t>(v >> 16));
+                        }
+                        // stage 0 of a tile always runs its residual MMAs (R starts there)
+                        has = g1 > g0 || i == 0;
                     }
-                    // stage 0 of a tile always runs its residual MMAs (R starts there)
-                    has = g1 > g0 || i == 0;
                     fence_proxy_async();  // the tile is read by the tensor core
                 }
                 if (lane == 0) rflag[4 * a + q] = has ? 1u : 0u;
@@ -544,7 +633,11 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     float v[32];
                     tmem_ld32(tl + T_D + b * BM + c0, v);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) acc[c0 + c] = fmaf(sc, v[c], acc[c0 + c]);
+                    for (int c = 0; c < 32; ++c) {
+                        // A4: an exact int32 group sum, at most 128 * 15 * 8 in magnitude
+                        const float d = A4 ? small_int_to_f32(__float_as_uint(v[c])) : v[c];
+                        acc[c0 + c] = fmaf(sc, d, acc[c0 + c]);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -562,7 +655,11 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     float v[32];
                     tmem_ld32(tl + T_R + c0, v);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) acc[c0 + c] = fmaf(sr, v[c], acc[c0 + c]);
+                    for (int c = 0; c < 32; ++c) {
+                        // A4: an exact int32 sum of at most K products of magnitude 64
+                        const float d = A4 ? small_int_to_f32(__float_as_uint(v[c])) : v[c];
+                        acc[c0 + c] = fmaf(sr, d, acc[c0 + c]);
+                    }
                 }
             }
             tc_fence_before();
@@ -576,6 +673,14 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
 #pragma unroll
                     for (int c = 0; c < EPI_TOK; ++c)
                         if (c < nt) yc[static_cast<size_t>(c) * p.N] = acc[c];
+                } else if (A4) {
+                    // Y = s_x[token] * (sum_g s_g D_g + s_r R); the token's scale is
+                    // the same for every lane of the warp
+                    __nv_bfloat16 *yc = p.Y + static_cast<size_t>(m0 + tb) * p.N + row;
+                    const float *xs = p.xscale + m0 + tb;
+#pragma unroll
+                    for (int c = 0; c < EPI_TOK; ++c)
+                        if (c < nt) yc[static_cast<size_t>(c) * p.N] = __float2bfloat16_rn(acc[c] * __ldg(xs + c));
                 } else {
                     __nv_bfloat16 *yc = p.Y + static_cast<size_t>(m0 + tb) * p.N + row;
 #pragma unroll
@@ -595,11 +700,17 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
 
 }  // namespace
 
-mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
-                         cudaStream_t stream, float *partial) {
+namespace {
+
+// The shared launch path: A4 takes int8 activation codes and their per-token
+// scales in place of bf16 X.
+template <bool A4>
+mq_status launch_prefill_impl(const mq_weight *w, const void *X, const float *xscale, int64_t M,
+                              void *Y, cudaStream_t stream, float *partial) {
     const DeviceWeight &d = weight_device(w);
     if (d.Gp > 256) return fail(MQ_ERR_UNSUPPORTED, "prefill kernel: K above 32768");
     if (M > (int64_t(1) << 23)) return fail(MQ_ERR_UNSUPPORTED, "prefill kernel: M above 2^23");
+    if (A4 && d.K % 256) return fail(MQ_ERR_UNSUPPORTED, "W4A4 prefill kernel: K must be a multiple of 256");
     const PrefillMaps *pm = prefill_maps(w);
     if (!pm) return MQ_ERR_CUDA;
     PrefillParams p;
@@ -607,8 +718,9 @@ mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
     // four stages per X copy; two when the residual tiles take their share of
     // shared memory (a deeper ring of smaller copies)
     p.CX = p.with_residual ? 2 : 4;
-    if (!encode_x_map(&p.tm_x, X, M, d.K, p.CX))
+    if (!(A4 ? encode_codes_map(&p.tm_x, X, M, d.K, p.CX) : encode_x_map(&p.tm_x, X, M, d.K, p.CX)))
         return fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for X");
+    p.xscale = xscale;
     p.tm_w = pm->w;
     p.pw = pm->pw;
     p.stage_ptr = d.stage_ptr;
@@ -640,9 +752,9 @@ mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
     if (dev < 0 || dev >= 64) return fail(MQ_ERR_UNSUPPORTED, "device ordinal above 63");
     if (!configured[dev]) {
-        if (cudaFuncSetAttribute(prefill_kernel<NSLOT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(prefill_kernel<NSLOT, A4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  227 * 1024) != cudaSuccess ||
-            cudaFuncSetAttribute(prefill_kernel<MAX_NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(prefill_kernel<MAX_NS, A4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  227 * 1024) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             sms[dev] <= 0)
@@ -652,13 +764,25 @@ mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
     // one CTA per SM (its shared memory and 512 TMEM columns allow no second)
     const int grid = static_cast<int>(std::min<int64_t>(tiles, sms[dev]));
     if (p.with_residual)
-        prefill_kernel<NSLOT><<<grid, THREADS, smem, stream>>>(p);
+        prefill_kernel<NSLOT, A4><<<grid, THREADS, smem, stream>>>(p);
     else
-        prefill_kernel<MAX_NS><<<grid, THREADS, smem, stream>>>(p);
+        prefill_kernel<MAX_NS, A4><<<grid, THREADS, smem, stream>>>(p);
     cudaError_t e = cudaPeekAtLastError();
     if (e != cudaSuccess)
         return fail(MQ_ERR_CUDA, std::string("prefill launch: ") + cudaGetErrorString(e));
     return MQ_OK;
+}
+
+}  // namespace
+
+mq_status launch_prefill(const mq_weight *w, const void *X, int64_t M, void *Y,
+                         cudaStream_t stream, float *partial) {
+    return launch_prefill_impl<false>(w, X, nullptr, M, Y, stream, partial);
+}
+
+mq_status launch_prefill_a4(const mq_weight *w, const int8_t *codes, const float *xscale, int64_t M,
+                            void *Y, cudaStream_t stream) {
+    return launch_prefill_impl<true>(w, codes, xscale, M, Y, stream, nullptr);
 }
 
 }  // namespace mq

@@ -267,9 +267,10 @@ class Weight:
         return Y
 
     def linear_w4a4(self, X, Y=None, workspace=None, *, stream=None):
-        """The W4A4 variant for M <= 16: per-token int4 activation codes in a
+        """The W4A4 variant: per-token int4 activation codes in a
         caller-owned workspace (mq_w4a4_workspace_bytes), then the fused
-        int4 x int4 pass."""
+        int4 x int4 pass (decode kernels for M <= 16, the tcgen05 prefill
+        kernel above, which needs K % 256 == 0)."""
         import torch
         info = self.info()
         X = X.contiguous()

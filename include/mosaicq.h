@@ -231,9 +231,11 @@ int64_t mq_w4a4_workspace_bytes(const mq_weight *w, int64_t M);
  * exact int32 group sums), the int4 x int4 residual and the scaling.
  * X, Y as for mq_linear; workspace: caller-owned device memory of at least
  * mq_w4a4_workspace_bytes(w, M) bytes, 16-byte aligned, not shared with a
- * concurrent call. Asynchronous, no allocation. M in [0, 16] (the decode
- * regime): UNSUPPORTED for M > 16. Errors as mq_linear, plus INVALID_ARG for
- * a NULL, misaligned or too small workspace. */
+ * concurrent call. Asynchronous, no allocation. M <= 16 runs the decode
+ * kernels (int8 mma.sync); larger M the prefill kernel (tcgen05 kind::i8
+ * MMAs into int32 in tensor memory), which needs K to be a multiple of 256:
+ * UNSUPPORTED otherwise, and for M above 2^23. Errors as mq_linear, plus
+ * INVALID_ARG for a NULL, misaligned or too small workspace. */
 mq_status mq_linear_w4a4(const mq_weight *w, const void *X_dev, int64_t M, void *Y_dev,
                          void *workspace, size_t workspace_bytes, mq_stream stream);
 

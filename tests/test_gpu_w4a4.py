@@ -86,10 +86,10 @@ def test_w4a4_7b_shapes_sampled_rows(mq, cuda):
 
 
 def test_w4a4_errors(mq, cuda):
-    W = synth.weight(64, 256, std=0.02, outlier_frac=0.01, seed=93)
+    W = synth.weight(64, 384, std=0.02, outlier_frac=0.01, seed=93)
     w = mq.Weight.pack(W, 0.02)
-    X = synth.activations(17, 256, seed=94).cuda()
-    with pytest.raises(mq.MQError) as e:
+    X = synth.activations(17, 384, seed=94).cuda()
+    with pytest.raises(mq.MQError) as e:      # the prefill form needs K % 256 == 0
         w.linear_w4a4(X)
     assert e.value.status == mq.UNSUPPORTED
     ws = torch.empty(16, dtype=torch.uint8, device="cuda")
@@ -129,4 +129,54 @@ def test_w4a4_70b_mlp_sampled_rows(mq, cuda):
                                      np.random.default_rng(1).choice(N, 48, replace=False)]))
     d = oracle.decompose(np.ascontiguousarray(W[rows]), rho)
     r = oracle_check_w4a4(Y[:, torch.from_numpy(rows).cuda()], X, d)
+    assert r["ok"], r
+
+
+# ---------------------------------------------------------------- M > 16: the tcgen05 prefill kernel (kind::i8)
+@pytest.mark.parametrize("N,K,M,rho", [
+    (512, 4096, 17, 0.005),      # one partial token tile
+    (300, 1024, 200, 0.02),      # ragged rows and tokens, two token tiles
+    (256, 2048, 256, 0.0),       # no residual: eight operand slots
+    (384, 512, 130, 0.05),       # dense residual, a 2-token last tile
+    (128, 8192, 64, 0.01),       # long K
+    (1000, 768, 129, 0.005),     # 6 groups, ragged rows
+])
+def test_w4a4_prefill_parity(mq, cuda, N, K, M, rho):
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=N + K + M)
+    X = synth.activations(M, K, seed=M + 7, channels=4, mult=20.0)
+    X[M // 2] = 0                                 # a zero token: scale 1, output 0
+    w = mq.Weight.pack(W, rho)
+    Y = w.linear_w4a4(X.cuda())
+    torch.cuda.synchronize()
+    assert w.device_error() == 0
+    assert not Y[M // 2].any()
+    r = oracle_check_w4a4(Y, X, oracle.decompose(W, rho))
+    assert r["ok"], r
+
+
+def test_w4a4_prefill_block_residual(mq, cuda):
+    W = synth.weight(256, 4096, std=0.02, outlier_frac=0.005, seed=95)
+    w = mq.Weight.pack(W, block_fraction=0.25)
+    X = synth.activations(100, 4096, seed=96, channels=4, mult=20.0)
+    Y = w.linear_w4a4(X.cuda())
+    torch.cuda.synchronize()
+    assert w.device_error() == 0
+    r = oracle_check_w4a4(Y, X, oracle.decompose_blocks(W, 0.25))
+    assert r["ok"], r
+
+
+def test_w4a4_prefill_full_size_sampled_rows(mq, cuda):
+    # the prefill workload (M = 2048, 14336 x 4096, density 0.5 %) in the
+    # launch configuration the bench times, 64 rows against the oracle
+    W, X, rho = synth.workload_inputs("prefill")
+    N = W.shape[0]
+    w = mq.Weight.pack(W, rho)
+    Y = w.linear_w4a4(X.cuda())
+    torch.cuda.synchronize()
+    assert w.device_error() == 0
+    rows = np.unique(np.concatenate([np.arange(0, 16), np.arange(N - 16, N),
+                                     np.random.default_rng(3).choice(N, 32, replace=False)]))
+    d = oracle.decompose(np.ascontiguousarray(W[rows]), rho)
+    sub = Y[:, torch.from_numpy(rows).cuda()]
+    r = oracle_check_w4a4(sub, X, d)
     assert r["ok"], r
