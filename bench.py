@@ -715,11 +715,14 @@ def run_distortion():
 # ------------------------------------------------------------------ W4A4
 def run_w4a4():
     """The W4A4 variant against W4A16 on the same packed weights: the three
-    7B decode shapes at M = 1 and the 70B MLP at M = 16. Each path is timed as
-    a CUDA graph of 48 back-to-back calls, weights rotated through copies
-    larger than L2 (the W4A4 call is two launches: quantization, then the
-    fused product). Bytes are the algorithmic bytes of the W4A16 call (packed
-    weight, CSR, bf16 X and Y once). Prints one JSON line."""
+    7B decode shapes at M = 1, the 70B MLP at M = 16 and the prefill
+    workload at M = 2048. Each path is timed as a CUDA graph of 48
+    back-to-back calls, weights rotated through copies larger than L2 (the
+    W4A4 call is two launches: quantization, then the fused product). Bytes
+    are the algorithmic bytes of the W4A16 call (packed weight, CSR, bf16 X
+    and Y once); at M > 16 the line also gives TFLOP/s against the tensor
+    peak of the call's MMA kind (bf16 measured; int8 = 2 x the measured bf16
+    figure, the nominal dense ratio). Prints one JSON line."""
     import torch
     from bit_gemm_w4_b200 import mosaicq as mq, synth
     dev = torch.device("cuda:0")
@@ -728,7 +731,7 @@ def run_w4a4():
     pk, _ = peaks()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     rows = []
-    for name in ("7b_decode", "70b_mlp"):
+    for name in ("7b_decode", "70b_mlp", "prefill"):
         cfg = synth.WORKLOADS[name]
         for i, (N, K) in enumerate(cfg["shapes"]):
             per = alg_bytes(cfg["M"], N, K, 0)
@@ -777,6 +780,11 @@ def run_w4a4():
                 by = alg_bytes(M, N, K, nnz)
                 out[path] = {"us": round(us, 3), "TB_s": round(by / us / 1e6, 3),
                              "frac": round(by / us / 1e3 / pk["hbm_gbs"], 4)}
+                if M > 16:
+                    tf = alg_flops(M, N, K, nnz) / us / 1e6
+                    peak = pk["bf16_tflops"] * (2.0 if path == "w4a4" else 1.0)
+                    out[path].update({"TFLOP_s": round(tf, 1), "tensor_peak_tflops": round(peak, 1),
+                                      "tensor_frac": round(tf / peak, 4)})
                 del g
             rows.append(out)
             del ws
