@@ -360,6 +360,7 @@ def test_bounded_wait_gives_up(mq, cuda):
     (200, 384, 77, "prefill"),    # prefill, ragged tiles
     (200, 384, 5, "w4a4"),        # W4A4
     (19000, 384, 12, "w4a4"),     # W4A4 through the wide kernel
+    (200, 512, 77, "w4a4"),       # W4A4 through the prefill kernel, ragged tiles
 ])
 def test_outputs_stay_inside_y(mq, cuda, N, K, M, path):
     # Y lives inside a canary-filled buffer; only its M x N elements may change
