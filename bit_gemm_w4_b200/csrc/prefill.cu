@@ -477,15 +477,23 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     nb1 = __ldg(gptr + 5);
                 }
             }
-            // the scale / zero word of the next group is requested a group early,
-            // so its latency is not exposed behind waits that complete at once
-            uint32_t sz_next = valid ? __ldg(szrow) : 0u, szw = 0u;
+            // scale / zero words four groups per 16-byte load (rows are padded to a
+            // multiple of four groups), the next four requested when these are
+            // taken, so the loads are few and their latency is hidden
+            uint4 sz4 = make_uint4(0u, 0u, 0u, 0u);
+            uint4 sz4_next = valid ? __ldg(reinterpret_cast<const uint4 *>(szrow)) : sz4;
+            uint32_t szw = 0u;
             constexpr int SPG = A4 ? 1 : 2;  // stages per quantization group
             for (int i = 0, pi = 0; i < nk; ++i, ++it) {
                 const int a = it & (NS - 1), ps = pc & (NPSLOT - 1);
                 if (i % SPG == 0) {
-                    szw = sz_next;
-                    sz_next = (valid && i / SPG + 1 < G) ? __ldg(szrow + i / SPG + 1) : 0u;
+                    const int g = i / SPG;
+                    if ((g & 3) == 0) {
+                        sz4 = sz4_next;
+                        if (valid && g + 4 < Gp)
+                            sz4_next = __ldg(reinterpret_cast<const uint4 *>(szrow + g + 4));
+                    }
+                    szw = (g & 2) ? ((g & 1) ? sz4.w : sz4.z) : ((g & 1) ? sz4.y : sz4.x);
                 }
                 // this warp's residual group of the stage and its first entry per lane
                 const int g0 = na0, g1 = na1;
