@@ -569,6 +569,7 @@ PROFILE_CASES = {
     "prefill-14336x4096-m256": (14336, 4096, 256, 0.005, "prefill"),
     "prefill-14336x4096-m2048": (14336, 4096, 2048, 0.005, "prefill"),
     "prefill-14336x4096-m2048-dense": (14336, 4096, 2048, 0.0, "prefill"),
+    "prefill-w4a4-14336x4096-m2048": (14336, 4096, 2048, 0.005, "w4a4"),
 }
 
 
@@ -584,14 +585,22 @@ def run_profile_case(name: str, reps: int):
     W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=1)
     w = mq.Weight.pack(W, rho)
     X = synth.activations(M, K, seed=2, channels=8, mult=30.0).to(dev)
-    Y = w.linear(X, path=path)
+    ws = None
+    if path == "w4a4":  # activation quantization, then the fused W4A4 pass
+        ws = torch.empty(int(mq._lib.mq_w4a4_workspace_bytes(w._h, M)), dtype=torch.uint8, device=dev)
+        Y = w.linear_w4a4(X, workspace=ws)
+    else:
+        Y = w.linear(X, path=path)
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
     ts = []
     for _ in range(reps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        w.linear(X, Y, path=path)
+        if ws is not None:
+            w.linear_w4a4(X, Y, ws)
+        else:
+            w.linear(X, Y, path=path)
         b.record()
         torch.cuda.synchronize()
         ts.append(a.elapsed_time(b) * 1e3)
