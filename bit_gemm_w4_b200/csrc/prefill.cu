@@ -46,6 +46,16 @@
 // MMAs run meanwhile into the other buffer. After a tile's last stage R is
 // scaled by s_r[n] and added (the reduction-add) and the tile is stored as
 // bf16, while the next tile's MMAs already run.
+// Without a residual, R's 128 columns hold four more operand slots (eight).
+//
+// W4A4 form (the pipeline's quantization stage in front, per-token int4
+// activation codes): X is the int8 codes, each 8-column chunk already in the
+// packed codes' k order, and a stage is 128 columns, one quantization group,
+// so the X tile and the operand slot keep their sizes. The dequant warps write
+// int8 codes q - z (a carry-free byte subtraction), the MMAs are kind::i8
+// (s8 x s8 -> s32, exact) and every stage commits its own group partial; the
+// epilogue converts the int32 sums to fp32 exactly, applies s[n][g] and s_r[n]
+// and multiplies by the token's scale s_x when it stores Y.
 
 #include "common.cuh"
 #include "internal.h"
