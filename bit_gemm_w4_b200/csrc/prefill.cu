@@ -476,15 +476,22 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
             // The residual entries are requested ahead of use: a stage's group
             // bounds two stages early, its first entry per lane one stage early,
             // so neither global load sits on the path from the waits to the MMA.
-            int na0 = 0, na1 = 0, nb0 = 0, nb1 = 0;
-            uint32_t nv = 0u;
-            if (!A4 && res) {
-                na0 = __ldg(gptr);
-                na1 = __ldg(gptr + 1);
-                if (na0 + lane < na1) nv = __ldg(p.stage_ent + na0 + lane);
-                if (nk > 1) {
-                    nb0 = __ldg(gptr + 4);
-                    nb1 = __ldg(gptr + 5);
+            // A stage holds NSUB of the 64-column lists (two for A4's 128 columns).
+            constexpr int NSUB = A4 ? 2 : 1;
+            int na[NSUB][2], nb[NSUB][2];
+            uint32_t nv[NSUB];
+#pragma unroll
+            for (int u = 0; u < NSUB; ++u) {
+                na[u][0] = na[u][1] = nb[u][0] = nb[u][1] = 0;
+                nv[u] = 0u;
+                if (res) {
+                    na[u][0] = __ldg(gptr + 4 * u);
+                    na[u][1] = __ldg(gptr + 4 * u + 1);
+                    if (na[u][0] + lane < na[u][1]) nv[u] = __ldg(p.stage_ent + na[u][0] + lane);
+                    if (nk > 1) {
+                        nb[u][0] = __ldg(gptr + 4 * (NSUB + u));
+                        nb[u][1] = __ldg(gptr + 4 * (NSUB + u) + 1);
+                    }
                 }
             }
             // scale / zero words four groups per 16-byte load (rows are padded to a
@@ -505,16 +512,23 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     }
                     szw = (g & 2) ? ((g & 1) ? sz4.w : sz4.z) : ((g & 1) ? sz4.y : sz4.x);
                 }
-                // this warp's residual group of the stage and its first entry per lane
-                const int g0 = na0, g1 = na1;
-                const uint32_t v0 = nv;
-                if (!A4 && res) {
-                    na0 = nb0;
-                    na1 = nb1;
-                    nv = (i + 1 < nk && na0 + lane < na1) ? __ldg(p.stage_ent + na0 + lane) : 0u;
-                    if (i + 2 < nk) {
-                        nb0 = __ldg(gptr + 4 * (i + 2));
-                        nb1 = __ldg(gptr + 4 * (i + 2) + 1);
+                // this warp's residual groups of the stage and their first entries per lane
+                int g[NSUB][2];
+                uint32_t v0[NSUB];
+#pragma unroll
+                for (int u = 0; u < NSUB; ++u) {
+                    g[u][0] = na[u][0];
+                    g[u][1] = na[u][1];
+                    v0[u] = nv[u];
+                    if (res) {
+                        na[u][0] = nb[u][0];
+                        na[u][1] = nb[u][1];
+                        nv[u] = (i + 1 < nk && na[u][0] + lane < na[u][1])
+                                    ? __ldg(p.stage_ent + na[u][0] + lane) : 0u;
+                        if (i + 2 < nk) {
+                            nb[u][0] = __ldg(gptr + 4 * (NSUB * (i + 2) + u));
+                            nb[u][1] = __ldg(gptr + 4 * (NSUB * (i + 2) + u) + 1);
+                        }
                     }
                 }
                 if ((pi == 0 &&
@@ -582,35 +596,28 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                             sts128(rq + 512 * k + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
                     }
                     __syncwarp();
-                    if constexpr (A4) {
-                        // the two 64-column list stages of this 128-column stage; an
-                        // int8 code goes to its column's position in the chunk's order
-                        int cnt = 0;
+                    int cnt = 0;
 #pragma unroll
-                        for (int sub = 0; sub < 2; ++sub) {
-                            const int e0 = __ldg(gptr + 4 * (2 * i + sub));
-                            const int e1 = __ldg(gptr + 4 * (2 * i + sub) + 1);
-                            cnt += e1 - e0;
-                            for (int e = e0 + lane; e < e1; e += 32) {
-                                const uint32_t v = __ldg(p.stage_ent + e);
-                                const int r = v & 127, c = ((v >> 8) & 63) + 64 * sub;
+                    for (int u = 0; u < NSUB; ++u) {
+                        cnt += g[u][1] - g[u][0];
+                        for (int e = g[u][0] + lane; e < g[u][1]; e += 32) {
+                            const uint32_t v = (e == g[u][0] + lane) ? v0[u] : __ldg(p.stage_ent + e);
+                            const int r = v & 127, c = ((v >> 8) & 63) + 64 * u;
+                            if constexpr (A4) {
+                                // an int8 code goes to its column's position in the
+                                // chunk's code order
                                 const int cp = (c & ~7) | ((c & 3) << 1) | ((c >> 2) & 1);
                                 const int q8 = static_cast<int>(bf16_bits_to_f32(v >> 16));
                                 sts_u8(rt + r * 128 + (((cp >> 4) ^ (r & 7)) << 4) + (cp & 15),
                                        static_cast<uint8_t>(q8 & 0xFF));
+                            } else {
+                                sts16(rt + r * 128 + (((c >> 3) ^ (r & 7)) << 4) + (c & 7) * 2,
+                                      static_cast<uint16_t>(v >> 16));
                             }
                         }
-                        has = cnt > 0 || i == 0;
-                    } else {
-                        for (int e = g0 + lane; e < g1; e += 32) {
-                            const uint32_t v = (e == g0 + lane) ? v0 : __ldg(p.stage_ent + e);
-                            const int r = v & 127, c = (v >> 8) & 63;
-                            sts16(rt + r * 128 + (((c >> 3) ^ (r & 7)) << 4) + (c & 7) * 2,
-                                  static_cast<uint16_t>(v >> 16));
-                        }
-                        // stage 0 of a tile always runs its residual MMAs (R starts there)
-                        has = g1 > g0 || i == 0;
                     }
+                    // stage 0 of a tile always runs its residual MMAs (R starts there)
+                    has = cnt > 0 || i == 0;
                     fence_proxy_async();  // the tile is read by the tensor core
                 }
                 if (lane == 0) rflag[4 * a + q] = has ? 1u : 0u;
