@@ -32,9 +32,10 @@
 //               tcgen05.st. The row's residual entries of the stage are
 //               scattered as exact bf16 codes q_r into a shared-memory tile
 //               (128-byte swizzle, K-major) that is otherwise zero; when the
-//               slot comes round again only those entries are cleared.
+//               slot comes round again the warp zeroes its 32 rows of it.
 // Tensor memory (512 columns): the group partials D[2] at 0 / 128, the
-// residual accumulator R at 256, four 32-column operand slots at 384.
+// residual accumulator R at 256 and four 32-column operand slots at 384, or,
+// without a residual, eight operand slots at 256.
 // Per stage the MMA thread issues 4 K=16 steps of the dense codes (A from
 // tensor memory) into the TMEM buffer of the current 128-column group and,
 // when any of the tile's rows has a residual entry in the stage, 4 steps of
@@ -46,7 +47,6 @@
 // MMAs run meanwhile into the other buffer. After a tile's last stage R is
 // scaled by s_r[n] and added (the reduction-add) and the tile is stored as
 // bf16, while the next tile's MMAs already run.
-// Without a residual, R's 128 columns hold four more operand slots (eight).
 //
 // W4A4 form (the pipeline's quantization stage in front, per-token int4
 // activation codes): X is the int8 codes, each 8-column chunk already in the
