@@ -72,6 +72,7 @@ def _load():
         "mq_free": ([vp], None),
         "mq_residual_nnz": ([i64, i64, ctypes.POINTER(_PackOpts), ctypes.POINTER(i64)], st),
         "mq_pack_host": ([vp, i64, i64, ctypes.POINTER(_PackOpts), ctypes.POINTER(_HostPacked)], st),
+        "mq_prefill_lists_host": ([i64, i64, vp, vp, vp, vp, vp], st),
         "mq_pack_decomposed": ([ctypes.POINTER(_Decomp), vp, ctypes.POINTER(vp)], st),
         "mq_get_info": ([vp, ctypes.POINTER(_Info)], st),
         "mq_export": ([vp, ctypes.POINTER(_HostPacked)], st),
@@ -152,6 +153,20 @@ def pack_host(W: np.ndarray, rho: float, group: int = 128, *, block_fraction=Non
     _check(_lib.mq_pack_host(_ptr(W), N, K, ctypes.byref(o), ctypes.byref(hp)), "mq_pack_host")
     del keep
     return arrs
+
+
+def prefill_lists_host(N: int, K: int, packed: dict):
+    """The prefill kernel's residual lists of a host pack (pack_host's arrays):
+    (ptr int32 [ceil(N/128) * K/64 * 4 + 1], ent uint32 [nnz]); no CUDA call."""
+    row_ptr = np.ascontiguousarray(packed["row_ptr"], np.int32)
+    col = np.ascontiguousarray(packed["col"], np.uint16)
+    val = np.ascontiguousarray(packed["val"], np.uint8)
+    nnz = int(row_ptr[-1])
+    ptr = np.zeros(((N + 127) // 128) * (K // 64) * 4 + 1, np.int32)
+    ent = np.zeros(max(nnz, 1), np.uint32)
+    _check(_lib.mq_prefill_lists_host(N, K, _ptr(row_ptr), _ptr(col), _ptr(val), _ptr(ptr), _ptr(ent)),
+           "mq_prefill_lists_host")
+    return ptr, ent[:nnz]
 
 
 def selftest_bounded_wait(limit_cycles: int = 1 << 20) -> list:

@@ -266,6 +266,17 @@ mq_status mq_residual_nnz(int64_t N, int64_t K, const mq_pack_opts *opts,
 mq_status mq_pack_host(const float *W_host, int64_t N, int64_t K,
                        const mq_pack_opts *opts, mq_host_packed *out);
 
+/* Test support, no CUDA call: the residual of a host pack regrouped as the
+ * prefill kernel reads it. row_ptr [N+1], col [nnz], val [(nnz+1)/2] are the
+ * packed CSR (mq_pack_host) of an N x K weight, K a multiple of 64. Writes
+ * ptr: int32 [ceil(N/128) * (K/64) * 4 + 1], the first entry of each
+ * (128-row tile, 64-column stage, 32-row quadrant) group in that order, and
+ * ent: uint32 [nnz], each entry as row-in-tile | column-in-stage << 8 |
+ * bf16 bits of q_r << 16, ordered by (group, row, column). INVALID_ARG for
+ * a bad shape, NULL buffers, a malformed row_ptr or a column not below K. */
+mq_status mq_prefill_lists_host(int64_t N, int64_t K, const int32_t *row_ptr, const uint16_t *col,
+                                const uint8_t *val, int32_t *ptr, uint32_t *ent);
+
 /* Pack a given decomposition (validated: code ranges, integer zero points
  * 0..15, finite scales, CSR structure) and upload it like mq_pack. */
 mq_status mq_pack_decomposed(const mq_decomp *d, mq_stream stream,

@@ -1,0 +1,69 @@
+"""The prefill kernel's residual lists, built on the host at upload, checked
+on the CPU: regrouping the packed CSR by (128-row tile, 64-column stage,
+32-row quadrant) must give back every entry exactly once, with its row,
+column and int4 code, in (group, row, column) order (mq_prefill_lists_host
+exports the lists the upload sends to the device)."""
+
+import numpy as np
+import pytest
+
+from bit_gemm_w4_b200 import mosaicq as mq, synth
+
+
+def _entries(packed):
+    """(row, column, code) of every CSR entry of a host pack."""
+    rp, col, val = packed["row_ptr"], packed["col"], packed["val"]
+    out = []
+    for n in range(len(rp) - 1):
+        for e in range(rp[n], rp[n + 1]):
+            nib = (int(val[e >> 1]) >> ((e & 1) * 4)) & 0xF
+            out.append((n, int(col[e]), (nib ^ 8) - 8))
+    return out
+
+
+def _expected(N, K, packed):
+    nk = K // 64
+    keys = ((N + 127) // 128) * nk * 4
+    groups = [[] for _ in range(keys)]
+    for n, c, q in _entries(packed):
+        groups[((n // 128) * nk + c // 64) * 4 + (n % 128) // 32].append((n, c, q))
+    ptr = np.zeros(keys + 1, np.int64)
+    ent = []
+    for k, g in enumerate(groups):
+        g.sort()
+        ptr[k + 1] = ptr[k] + len(g)
+        for n, c, q in g:
+            bits = int(np.array([q], np.float32).view(np.uint32)[0]) & 0xFFFF0000
+            ent.append((n % 128) | ((c % 64) << 8) | bits)
+    return ptr, np.array(ent, np.uint64)
+
+
+@pytest.mark.parametrize("N,K,rho,blocks", [
+    (300, 512, 0.05, None),      # ragged last tile, row mode
+    (128, 384, 0.1, None),       # one tile, six stages
+    (256, 1024, 0.0, 0.25),      # block mode
+    (64, 256, 0.0, None),        # no residual
+])
+def test_prefill_lists_regroup_the_csr(N, K, rho, blocks):
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.01, seed=N + K)
+    packed = mq.pack_host(W, rho, block_fraction=blocks)
+    ptr, ent = mq.prefill_lists_host(N, K, packed)
+    eptr, eent = _expected(N, K, packed)
+    assert np.array_equal(ptr.astype(np.int64), eptr)
+    assert np.array_equal(ent.astype(np.uint64), eent)
+    # every code is an exact bf16 integer in [-8, 7]
+    codes = (ent.astype(np.uint32) & 0xFFFF0000).view(np.float32)
+    assert np.all(codes == np.round(codes)) and codes.min(initial=0) >= -8 and codes.max(initial=0) <= 7
+
+
+def test_prefill_lists_reject_bad_input():
+    rp = np.array([0, 2, 1], np.int32)           # decreasing offsets
+    packed = dict(row_ptr=rp, col=np.array([0, 1], np.uint16), val=np.array([0x12], np.uint8))
+    with pytest.raises(mq.MQError) as e:
+        mq.prefill_lists_host(2, 128, packed)
+    assert e.value.status == mq.INVALID_ARG
+    packed = dict(row_ptr=np.array([0, 1], np.int32), col=np.array([130], np.uint16),
+                  val=np.array([0x01], np.uint8))   # a column not below K
+    with pytest.raises(mq.MQError) as e:
+        mq.prefill_lists_host(1, 128, packed)
+    assert e.value.status == mq.INVALID_ARG
