@@ -400,6 +400,34 @@ mq_status mq_prefill_lists_host(int64_t N, int64_t K, const int32_t *row_ptr, co
     return MQ_OK;
 }
 
+mq_status mq_wide_lists_host(int64_t N, int64_t K, const int32_t *row_ptr, const uint16_t *col,
+                             const uint8_t *val, int32_t *ptr, uint16_t *off, uint16_t *ent,
+                             int64_t *max_len) {
+    if (N <= 0 || K <= 0 || K % 128) return fail(MQ_ERR_INVALID_ARG, "N, K: positive, K a multiple of 128");
+    if (!row_ptr || !ptr || !off || !max_len) return fail(MQ_ERR_INVALID_ARG, "a buffer is NULL");
+    const int64_t nnz = row_ptr[N];
+    if (row_ptr[0] != 0 || nnz < 0) return fail(MQ_ERR_INVALID_ARG, "row_ptr must start at 0");
+    for (int64_t n = 0; n < N; ++n)
+        if (row_ptr[n + 1] < row_ptr[n]) return fail(MQ_ERR_INVALID_ARG, "row_ptr must not decrease");
+    if (nnz > 0 && (!col || !val || !ent)) return fail(MQ_ERR_INVALID_ARG, "col, val or ent is NULL");
+    for (int64_t e = 0; e < nnz; ++e)
+        if (col[e] >= K) return fail(MQ_ERR_INVALID_ARG, "a column is not below K");
+    HostPacked hp;
+    hp.N = N;
+    hp.K = K;
+    hp.nnz = nnz;
+    hp.row_ptr.assign(row_ptr, row_ptr + N + 1);
+    hp.col.assign(col, col + nnz);
+    hp.val.assign(val, val + (nnz + 1) / 2);
+    std::vector<int32_t> hptr;
+    std::vector<uint16_t> hoff, hent;
+    build_wide_lists(hp, hptr, hoff, hent, *max_len);
+    std::memcpy(ptr, hptr.data(), hptr.size() * 4);
+    std::memcpy(off, hoff.data(), hoff.size() * 2);
+    if (nnz) std::memcpy(ent, hent.data(), hent.size() * 2);
+    return MQ_OK;
+}
+
 mq_status mq_pack(const float *W_host, int64_t N, int64_t K, const mq_pack_opts *opts,
                   mq_stream stream, mq_weight **out) {
     if (!out) return fail(MQ_ERR_INVALID_ARG, "out is NULL");

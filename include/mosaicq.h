@@ -277,6 +277,20 @@ mq_status mq_pack_host(const float *W_host, int64_t N, int64_t K,
 mq_status mq_prefill_lists_host(int64_t N, int64_t K, const int32_t *row_ptr, const uint16_t *col,
                                 const uint8_t *val, int32_t *ptr, uint32_t *ent);
 
+/* Test support, no CUDA call: the residual of a host pack regrouped as the
+ * wide decode kernel reads it, per (128-row block, 256-column stage) slice
+ * (S = ceil(K/256) stages, K a multiple of 128). Inside a slice the entries
+ * are ordered by the sub-key (row % 128) / 16 * 16 + (column % 256) / 128 * 8
+ * + (column % 32) / 4 (warp tile, 128-column group, MMA k-step), then by row
+ * and column. Writes ptr: int32 [ceil(N/128) * S + 1] slice starts; off:
+ * uint16 [ceil(N/128) * S * 136], off[slice * 136 + u] (u = 0..128) the start
+ * of sub-key u inside the slice; ent: uint16 [nnz], each entry as
+ * column % 256 | (row % 16) << 8 | stored nibble << 12; *max_len the longest
+ * slice. Errors as mq_prefill_lists_host. */
+mq_status mq_wide_lists_host(int64_t N, int64_t K, const int32_t *row_ptr, const uint16_t *col,
+                             const uint8_t *val, int32_t *ptr, uint16_t *off, uint16_t *ent,
+                             int64_t *max_len);
+
 /* Pack a given decomposition (validated: code ranges, integer zero points
  * 0..15, finite scales, CSR structure) and upload it like mq_pack. */
 mq_status mq_pack_decomposed(const mq_decomp *d, mq_stream stream,

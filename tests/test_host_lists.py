@@ -67,3 +67,45 @@ def test_prefill_lists_reject_bad_input():
     with pytest.raises(mq.MQError) as e:
         mq.prefill_lists_host(1, 128, packed)
     assert e.value.status == mq.INVALID_ARG
+
+
+def _wide_expected(N, K, packed):
+    S = (K + 255) // 256
+    slices = ((N + 127) // 128) * S
+    buckets = [[[] for _ in range(128)] for _ in range(slices)]
+    rp, col, val = packed["row_ptr"], packed["col"], packed["val"]
+    for n in range(N):
+        for e in range(rp[n], rp[n + 1]):
+            c = int(col[e])
+            nib = (int(val[e >> 1]) >> ((e & 1) * 4)) & 0xF
+            u = ((n % 128) // 16) * 16 + ((c % 256) // 128) * 8 + (c % 32) // 4
+            buckets[(n // 128) * S + c // 256][u].append((n, c, (c % 256) | ((n % 16) << 8) | (nib << 12)))
+    ptr = np.zeros(slices + 1, np.int64)
+    off = np.zeros((slices, 136), np.int64)
+    ent = []
+    for k in range(slices):
+        pos = 0
+        for u in range(128):
+            off[k, u] = pos
+            b = sorted(buckets[k][u])
+            ent.extend(w for _, _, w in b)
+            pos += len(b)
+        off[k, 128] = pos
+        ptr[k + 1] = ptr[k] + pos
+    return ptr, off, np.array(ent, np.int64)
+
+
+@pytest.mark.parametrize("N,K,rho,blocks", [
+    (300, 640, 0.05, None),      # ragged block, a half last stage (K % 256 = 128)
+    (256, 1024, 0.0, 0.25),      # block mode
+    (128, 256, 0.0, None),       # no residual
+])
+def test_wide_lists_regroup_the_csr(N, K, rho, blocks):
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.01, seed=2 * N + K)
+    packed = mq.pack_host(W, rho, block_fraction=blocks)
+    ptr, off, ent, mx = mq.wide_lists_host(N, K, packed)
+    eptr, eoff, eent = _wide_expected(N, K, packed)
+    assert np.array_equal(ptr.astype(np.int64), eptr)
+    assert np.array_equal(off[:, :129].astype(np.int64), eoff[:, :129])
+    assert np.array_equal(ent.astype(np.int64), eent)
+    assert mx == int(np.diff(eptr).max(initial=0))
