@@ -69,7 +69,7 @@ def alg_bytes(M: int, N: int, K: int, nnz: int) -> int:
 # profiles/ gives the command). The bench's other shapes are scaled by their
 # packed size N*K, which the traffic follows (no re-reads). Set to None when
 # the decode kernel changes until it is captured again.
-DECODE_TRAFFIC_4096 = 9.196032e6
+DECODE_TRAFFIC_4096 = None
 
 
 def alg_flops(M: int, N: int, K: int, nnz: int) -> int:

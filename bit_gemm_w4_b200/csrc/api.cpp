@@ -29,6 +29,7 @@ struct mq_weight {
     std::vector<int32_t> host_row_ptr;  // for residual tile statistics
     mutable std::mutex maps_mu;
     mutable std::vector<std::pair<int, int64_t>> tile_nnz;  // (tile height, max entries)
+    mutable std::vector<std::pair<int, int64_t>> span_nnz;  // (CTA count, max entries)
     mutable mq::PrefillMaps *pmaps = nullptr;
     ~mq_weight() { delete pmaps; }
 };
@@ -269,6 +270,20 @@ int64_t max_tile_nnz(const mq_weight *w, int bn) {
         mx = std::max<int64_t>(mx, w->host_row_ptr[r1] - w->host_row_ptr[r]);
     }
     w->tile_nnz.emplace_back(bn, mx);
+    return mx;
+}
+
+int64_t max_span_nnz(const mq_weight *w, int64_t ntile, int parts) {
+    std::lock_guard<std::mutex> lock(w->maps_mu);
+    for (const auto &e : w->span_nnz)
+        if (e.first == parts) return e.second;
+    int64_t mx = 0;
+    for (int64_t b = 0; b < parts; ++b) {
+        const int64_t r0 = std::min<int64_t>(w->d.N, 16 * (ntile * b / parts));
+        const int64_t r1 = std::min<int64_t>(w->d.N, 16 * (ntile * (b + 1) / parts));
+        mx = std::max<int64_t>(mx, w->host_row_ptr[r1] - w->host_row_ptr[r0]);
+    }
+    w->span_nnz.emplace_back(parts, mx);
     return mx;
 }
 

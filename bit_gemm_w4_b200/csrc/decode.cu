@@ -454,6 +454,10 @@ mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaS
         const mq_status st = launch_decode_wide(w, X, M, Y, stream, partial, pf);
         if (st != MQ_ERR_UNSUPPORTED) return st;
     }
+    if (M <= 8) {
+        const mq_status st = launch_decode_stream(w, X, M, Y, stream, partial, pf);
+        if (st != MQ_ERR_UNSUPPORTED) return st;
+    }
     if (M == 1) {
         // More 16-row tiles than two 8-warp CTAs per SM hold at once: 4-warp
         // CTAs (four per SM) overlap their waves better (11008 x 4096:

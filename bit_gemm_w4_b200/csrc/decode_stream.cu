@@ -1,0 +1,532 @@
+// Streaming decode kernel: Y[M][N] = X[M][K] * W_hat^T for M <= 8, one
+// fused pass over the packed weight.
+//
+// MosaicQuant "Methodology" 3. (ZipperEngine): the sparse residual is
+// computed inside the dense 4-bit GEMM pass over the same activations, and
+// the dense and sparse parts meet in one reduction-add.
+//
+// At a few tokens the layer is a read of the packed weight, and a decode
+// step is a chain of such launches. The kernel is shaped so that the chain
+// streams HBM without gaps:
+//   * Persistent: one CTA per SM, each owning a contiguous run of NT or
+//     NT - 1 16-row tiles (NT <= 8, a template parameter), so a CTA's bytes
+//     are one contiguous stretch of every packed array.
+//   * Small footprint (256 threads, at most 128 registers, under 100 KB of
+//     shared memory for the 7B-sized layers), so the next launch's CTAs fit
+//     beside this one's. With programmatic dependent launch every CTA
+//     releases the next grid at its first instruction; the next layer's
+//     weight stream then runs while this layer computes and drains, and only
+//     its read of X waits for this grid.
+//   * Every thread prefetches its own share of the packed codes through a
+//     private ring of D groups x NT tiles of cp.async stages in shared memory
+//     (no barrier between threads; each thread waits for its own copies). A
+//     slot is refilled with the item D groups ahead as soon as it has been
+//     consumed; slots, tiles and the wait depth are all compile-time
+//     constants, so the stream costs a few instructions per item.
+//   * The run's scale/zero words, its CSR slice (row offsets, columns,
+//     codes) and X are copied into shared memory once.
+//   * Warp w takes groups w, w+8, ... : for each group it loads the X
+//     fragment once, then walks the run's tiles (its rows g and g+8, 16
+//     bytes of each), keeping one fp32 accumulator set per tile in
+//     registers. Each group's nibbles become exact bf16 codes q - z (a mask
+//     into the mantissa of 128.0, then a subtraction of 128 + z); mma.sync
+//     m16n8k16 sums the exact products in fp32 and the group's partial is
+//     scaled by s in fp32. Subtracting (128 + z) * sum(x) once per group
+//     instead would save the subtraction, but the fp32 sums of (128 + q) * x
+//     then lose about 1e-5 absolute to cancellation, more than the
+//     per-element tolerance allows on small outputs.
+//   * Residual: after the dense pass, each half-warp walks the CSR entries of
+//     one row per tile (16 lanes per row), gathers x[m][col] from shared
+//     memory and reduces with shuffles; s_r times the sum joins the
+//     reduction.
+//   * Reduction-add: the eight warps' partials and the residual meet in
+//     shared memory and are stored once as bf16.
+// The k order inside a group is permuted so that each thread's 16-byte load
+// of packed codes feeds its own mma fragments with no shuffles: k-step s'
+// (0..7) of thread (g, t) covers columns 32t + 4s' + {0,1} and 32t + 4s' +
+// {2,3}; X is read in the same order, so the sum over k is unchanged.
+// X rows in shared memory are 16 bytes longer than K columns and each
+// group's 16-byte chunks are permuted (chunk c sits at c ^ 2 * ((c >> 3) &
+// 1)); scale/zero rows are padded to an odd multiple of four words. Both
+// keep a warp's shared-memory loads on distinct banks.
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "kernels.h"
+
+namespace mq {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTMax = 8;     // most tiles per CTA (one accumulator set each)
+constexpr int kMaxSmem = 200 * 1024;
+constexpr int kCsrBudget = 24 * 1024;  // shared memory for a CTA's CSR slice
+
+// Groups of prefetch ahead for NT tiles per CTA: eight to ten items per
+// thread (64-80 KB per CTA in flight), or one group for NT > 5.
+__host__ __device__ constexpr int groups_ahead(int nt) {
+    return nt >= 6 ? 1 : nt >= 4 ? 2 : nt == 3 ? 3 : nt == 2 ? 4 : 8;
+}
+
+struct StreamParams {
+    const uint32_t *qweight;  // [N][K/8]
+    const uint32_t *sz;       // [N][Gp]
+    const __nv_bfloat16 *X;   // [M][K]
+    __nv_bfloat16 *Y;         // [M][N]
+    float *Yf;                // fp32 dense-only output (unfused path) or null
+    const int32_t *row_ptr;
+    const uint16_t *col;
+    const uint8_t *val;
+    const uint16_t *rscale;
+    int M, N, K, G, Gp;
+    int ntile;      // ceil(N / 16)
+    int csr_cap;    // most residual entries of a CTA's run; 0: no residual
+    // 0x43004300 (bf16x2 128.0, 128.0), passed at run time so that it sits in
+    // a register and each code pair costs one LOP3 (mask and OR)
+    uint32_t bias;
+    L2Prefetch pf;  // another weight, brought into L2 meanwhile
+};
+
+// scale/zero row stride in shared memory (words): Gp, or Gp + 4, whichever
+// is an odd multiple of four
+__host__ __device__ inline int sz_stride(int Gp) { return ((Gp >> 2) & 1) ? Gp : Gp + 4; }
+
+// Shared-memory layout (bytes), identical on host and device.
+struct StreamLayout {
+    int ring, x, xrs, szs, red, res, rsf, rp, col, val, total;
+    __host__ __device__ StreamLayout(int M, int K, int Gp, int csr_cap, int nt) {
+        ring = 0;                                              // [D * NT][2][kThreads][16 B]
+        x = ring + groups_ahead(nt) * nt * 2 * kThreads * 16;  // [M][xrs]
+        xrs = K * 2 + 16;
+        szs = x + (M * xrs + 15) / 16 * 16;                    // [NT * 16][sz_stride] words
+        red = szs + nt * 16 * sz_stride(Gp) * 4;               // [NT][warp][M][16] fp32
+        res = red + nt * kWarps * M * 16 * 4;                  // [NT][M][16] fp32
+        rsf = res + nt * M * 16 * 4;                           // [NT * 16] fp32 s_r
+        rp = rsf + nt * 16 * 4;                                // [NT * 16 + 1] i32
+        col = rp + (csr_cap > 0 ? (nt * 16 + 1) * 4 + 15 : 0) / 16 * 16;
+        val = col + (csr_cap > 0 ? csr_cap * 2 + 32 : 0);
+        total = val + (csr_cap > 0 ? csr_cap / 2 + 48 : 0);
+    }
+};
+
+// bf16x2 (128 + q_lo, 128 + q_hi) for the nibbles at bits [0,4) and [16,20)
+// of w, with the bias word in a register: one LOP3.
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, uint32_t bias) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(0x000F000F), "r"(bias));
+    return d;
+}
+
+// bf16x2 (128 + z, 128 + z) from a scale/zero word (fp16 s low, fp16 z high,
+// z an integer 0..15): adding 1024 in fp16 puts z in the low mantissa bits.
+__device__ __forceinline__ uint32_t zero_pair(uint32_t szw) {
+    uint32_t h;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(h) : "r"(szw), "r"(0x64006400u));
+    return (__byte_perm(h, 0, 0x3232) & 0x000F000Fu) | 0x43004300u;
+}
+
+// cp.async of 16 bytes, or of none (zero fill) when `live` is false.
+__device__ __forceinline__ void cp_async16_if(void *dst, const void *src, bool live) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(live ? 16 : 0)
+                 : "memory");
+}
+
+__device__ __forceinline__ int xchunk(int c) { return c ^ (((c >> 3) & 1) << 1); }
+
+// D += A * B, m16n8k16 bf16 -> fp32, as a pure function of its operands (not
+// volatile), so that the compiler may interleave independent items.
+__device__ __forceinline__ void mma_pure(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+
+template <int MX, int NT>
+__global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid_constant__ StreamParams p) {
+    constexpr int D = groups_ahead(NT);
+    constexpr int R = D * NT;  // ring slots (items) per thread
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int M = MX == 1 ? 1 : p.M, N = p.N, K = p.K, G = p.G;
+    const StreamLayout L(M, K, p.Gp, p.csr_cap, NT);
+    const int SZS = sz_stride(p.Gp);
+    const int t0 = static_cast<int>(static_cast<long long>(p.ntile) * blockIdx.x / gridDim.x);
+    const int t1 = static_cast<int>(static_cast<long long>(p.ntile) * (blockIdx.x + 1) / gridDim.x);
+    const int nt = t1 - t0;      // NT or NT - 1
+    const bool full = nt == NT;  // only tile NT - 1 can be missing
+    const int gpw = warp < G ? (G - warp + kWarps - 1) / kWarps : 0;  // groups of this warp
+    const bool resid = p.csr_cap > 0;
+
+    // ------------------------------------------------ the weight stream
+    // Row offsets (words) of this thread's rows g and g+8 in each tile, and
+    // its 16-byte column within a group.
+    uint32_t off0[NT], off1[NT];
+    const uint32_t wrow = static_cast<uint32_t>(K / 8);
+#pragma unroll
+    for (int k = 0; k < NT; ++k) {
+        off0[k] = static_cast<uint32_t>(min((t0 + k) * 16 + g, N - 1)) * wrow;
+        off1[k] = static_cast<uint32_t>(min((t0 + k) * 16 + g + 8, N - 1)) * wrow;
+    }
+    const uint32_t *qbase = p.qweight + warp * 16 + 4 * t;
+    uint8_t *ring = smem + L.ring + threadIdx.x * 16;
+    // item (group j of this warp, tile k) into ring slot s
+    // (items past the end copy nothing: a source size of 0 writes zeros, and
+    // the address stays in bounds)
+    auto issue = [&](int j, int k, int s) {
+        const bool live = j < gpw && (k + 1 < NT || full);
+        const uint32_t *src = qbase + min(j, gpw - 1) * (kWarps * 16);
+        cp_async16_if(ring + s * (2 * kThreads * 16), src + off0[k], live);
+        cp_async16_if(ring + s * (2 * kThreads * 16) + kThreads * 16, src + off1[k], live);
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int d = 0; d < D; ++d)
+#pragma unroll
+        for (int k = 0; k < NT; ++k) issue(d, k, d * NT + k);
+    pdl_launch_dependents();
+    if (threadIdx.x == 0) {
+        l2_prefetch_share(p.pf, blockIdx.x, gridDim.x);
+        // X into L2 ahead of the wait: L2 is coherent, so a write of X by the
+        // previous grid after this prefetch still reaches the reads below
+        const long long xb = static_cast<long long>(M) * K * 2;
+        for (long long o = 0; o < xb; o += 1 << 16) {
+            const unsigned n = static_cast<unsigned>(xb - o < (1 << 16) ? xb - o : (1 << 16));
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<const char *>(p.X) + o), "r"(n)
+                         : "memory");
+        }
+    }
+
+    // ------------------------------------------------ the run's scale/zero words and CSR slice
+    const int n_lo = t0 * 16, n_hi = min(t1 * 16, N);
+    {
+        const int q4 = p.Gp / 4;  // 16-byte chunks per scale/zero row
+        for (int i = threadIdx.x; i < (n_hi - n_lo) * q4; i += kThreads) {
+            const int r = i / q4, q = i - r * q4;
+            cp_async16(smem + L.szs + (r * SZS + 4 * q) * 4,
+                       p.sz + static_cast<size_t>(n_lo + r) * p.Gp + 4 * q);
+        }
+    }
+    int col_base = 0, val_base = 0;
+    if (resid) {
+        for (int i = threadIdx.x; i <= n_hi - n_lo; i += kThreads)
+            cp_async4(smem + L.rp + 4 * i, p.row_ptr + n_lo + i);
+        const int e_lo = p.row_ptr[n_lo], e_hi = p.row_ptr[n_hi];
+        col_base = e_lo & ~7;
+        val_base = (e_lo >> 1) & ~15;
+        const int ncol16 = ((e_hi - col_base) * 2 + 15) / 16;
+        const int nval16 = (((e_hi + 1) >> 1) - val_base + 15) / 16;
+        for (int i = threadIdx.x; i < ncol16; i += kThreads)
+            cp_async16(smem + L.col + 16 * i, p.col + col_base + 8 * i);
+        for (int i = threadIdx.x; i < nval16; i += kThreads)
+            cp_async16(smem + L.val + 16 * i, p.val + val_base + 16 * i);
+    }
+    cp_async_commit();
+    if (resid)
+        for (int i = threadIdx.x; i < n_hi - n_lo; i += kThreads)
+            reinterpret_cast<float *>(smem + L.rsf)[i] = half_bits_to_f32(p.rscale[n_lo + i]);
+
+    // ------------------------------------------------ X
+    pdl_wait();  // X may come from the previous kernel; Y may still be read by it
+    {
+        const int chunks = K / 8;  // 16-byte chunks per token row
+        for (int m = 0; m < M; ++m)
+            for (int c = threadIdx.x; c < chunks; c += kThreads)
+                cp_async16(smem + L.x + m * L.xrs + (c >> 4) * 256 + xchunk(c & 15) * 16,
+                           p.X + static_cast<size_t>(m) * K + 8 * c);
+        cp_async_commit();
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    const uint8_t *xs = smem + L.x;
+    const uint32_t *szs = reinterpret_cast<const uint32_t *>(smem + L.szs);
+    float *red = reinterpret_cast<float *>(smem + L.red);
+    float *res = reinterpret_cast<float *>(smem + L.res);
+
+    // ------------------------------------------------ dense pass
+    float acc[NT][4];
+#pragma unroll
+    for (int k = 0; k < NT; ++k)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[k][i] = 0.f;
+    uint32_t xb[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) xb[i] = 0u;
+    const bool xlane = MX == 1 ? g == 0 : g < M;  // lanes whose token column is live
+#pragma unroll 1
+    for (int j0 = 0; j0 < gpw; j0 += D) {
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+            const int j = j0 + d;
+            if (j < gpw) {
+                const int gi = warp + kWarps * j;
+                if (xlane) {
+                    const uint8_t *xp = xs + g * L.xrs + gi * 256;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(xp + xchunk(4 * t + i) * 16);
+                        xb[4 * i + 0] = v.x;
+                        xb[4 * i + 1] = v.y;
+                        xb[4 * i + 2] = v.z;
+                        xb[4 * i + 3] = v.w;
+                    }
+                }
+                // one item: tile k of group gi, from ring slot d * NT + k
+                auto item = [&](int k) {
+                    const uint8_t *src = ring + (d * NT + k) * (2 * kThreads * 16);
+                    const uint4 wa = *reinterpret_cast<const uint4 *>(src);
+                    const uint4 wb = *reinterpret_cast<const uint4 *>(src + kThreads * 16);
+                    const uint32_t sz0 = szs[(k * 16 + g) * SZS + gi];
+                    const uint32_t sz1 = szs[(k * 16 + g + 8) * SZS + gi];
+                    const uint32_t zz0 = zero_pair(sz0), zz1 = zero_pair(sz1);
+                    const uint32_t bias = p.bias;
+                    // two accumulator chains (even and odd k-steps)
+                    float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+                    const uint32_t wr0[4] = {wa.x, wa.y, wa.z, wa.w};
+                    const uint32_t wr1[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t a_lo = wr0[ks >> 1] >> (8 * (ks & 1));
+                        const uint32_t b_lo = wr1[ks >> 1] >> (8 * (ks & 1));
+                        uint32_t a[4];
+                        a[0] = bf16x2_sub(nib_pair(a_lo, bias), zz0);
+                        a[1] = bf16x2_sub(nib_pair(b_lo, bias), zz1);
+                        a[2] = bf16x2_sub(nib_pair(a_lo >> 4, bias), zz0);
+                        a[3] = bf16x2_sub(nib_pair(b_lo >> 4, bias), zz1);
+                        if (ks & 1)
+                            mma_pure(cb, a, xb[2 * ks], xb[2 * ks + 1]);
+                        else
+                            mma_pure(ca, a, xb[2 * ks], xb[2 * ks + 1]);
+                    }
+                    const float s0 = half_bits_to_f32(sz0), s1 = half_bits_to_f32(sz1);
+                    acc[k][0] = fmaf(s0, ca[0] + cb[0], acc[k][0]);
+                    acc[k][2] = fmaf(s1, ca[2] + cb[2], acc[k][2]);
+                    if (MX > 1) {  // token columns 2t + 1 (none live at one token)
+                        acc[k][1] = fmaf(s0, ca[1] + cb[1], acc[k][1]);
+                        acc[k][3] = fmaf(s1, ca[3] + cb[3], acc[k][3]);
+                    }
+                };
+                // items in pairs after one wait, so that the two interleave;
+                // each slot is refilled D groups ahead once its values are used
+#pragma unroll
+                for (int k = 0; k < NT; k += 2) {
+                    if (k + 1 < NT) {
+                        cp_async_wait_group<R - 2>();
+                        item(k);
+                        if (k + 2 < NT || full) item(k + 1);
+                        issue(j + D, k, d * NT + k);
+                        issue(j + D, k + 1, d * NT + k + 1);
+                    } else {
+                        cp_async_wait_group<R - 1>();
+                        if (full) item(k);
+                        issue(j + D, k, d * NT + k);
+                    }
+                }
+            }
+        }
+    }
+    // this warp's partial sums: red[k][warp][m][row]
+#pragma unroll
+    for (int k = 0; k < NT; ++k) {
+        if (k < nt) {
+            float *rw = red + ((k * kWarps + warp) * M) * 16;
+            if (2 * t < M) {
+                rw[(2 * t) * 16 + g] = acc[k][0];
+                rw[(2 * t) * 16 + g + 8] = acc[k][2];
+            }
+            if (MX > 1 && 2 * t + 1 < M) {
+                rw[(2 * t + 1) * 16 + g] = acc[k][1];
+                rw[(2 * t + 1) * 16 + g + 8] = acc[k][3];
+            }
+        }
+    }
+
+    // ------------------------------------------------ residual: one row per half-warp and tile
+    if (resid) {
+        const int32_t *rps = reinterpret_cast<const int32_t *>(smem + L.rp);
+        const uint16_t *cols = reinterpret_cast<const uint16_t *>(smem + L.col);
+        const uint8_t *vals = smem + L.val;
+        const int rl = lane & 15, hw = 2 * warp + (lane >> 4);
+        const float *rsf = reinterpret_cast<const float *>(smem + L.rsf);
+        // q_r * x[m][c] for entry e of the staged slice
+        auto entry = [&](int e, float (&r)[MX]) {
+            const int cl = cols[e - col_base];
+            const uint32_t byte = vals[(e >> 1) - val_base];
+            const float q = static_cast<float>(static_cast<int>(((byte >> ((e & 1) * 4)) & 0xF) ^ 8) - 8);
+            const uint16_t *xe = reinterpret_cast<const uint16_t *>(
+                xs + (cl >> 7) * 256 + xchunk((cl & 127) >> 3) * 16 + (cl & 7) * 2);
+#pragma unroll
+            for (int m = 0; m < MX; ++m)
+                if (MX == 1 || m < M) r[m] = fmaf(q, bf16_bits_to_f32(xe[m * (L.xrs / 2)]), r[m]);
+        };
+        if constexpr (MX == 1) {
+            // one token: the rows of all tiles at once, so that their shared-
+            // memory reads overlap; the first two entries of each lane inline,
+            // longer rows in a loop
+            int a[NT], b[NT];
+            float r[NT][1];
+#pragma unroll
+            for (int k = 0; k < NT; ++k) {
+                const int row = (t0 + k) * 16 + hw;
+                const bool ok = (k + 1 < NT || full) && row < N;
+                a[k] = ok ? rps[row - n_lo] : 0;
+                b[k] = ok ? rps[row - n_lo + 1] : 0;
+                r[k][0] = 0.f;
+                if (a[k] + rl < b[k]) entry(a[k] + rl, r[k]);
+                if (a[k] + rl + 16 < b[k]) entry(a[k] + rl + 16, r[k]);
+            }
+#pragma unroll
+            for (int k = 0; k < NT; ++k)
+#pragma unroll 1
+                for (int e = a[k] + rl + 32; e < b[k]; e += 16) entry(e, r[k]);
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1)
+#pragma unroll
+                for (int k = 0; k < NT; ++k) r[k][0] += __shfl_xor_sync(0xffffffffu, r[k][0], off);
+            if (rl == 0) {
+#pragma unroll
+                for (int k = 0; k < NT; ++k) {
+                    const int row = (t0 + k) * 16 + hw;
+                    if (k + 1 < NT || full) res[k * 16 + hw] = b[k] > a[k] ? rsf[row - n_lo] * r[k][0] : 0.f;
+                }
+            }
+        } else {
+#pragma unroll 1
+            for (int k = 0; k < nt; ++k) {
+                const int row = (t0 + k) * 16 + hw;
+                int a = 0, b = 0;
+                if (row < N) {
+                    a = rps[row - n_lo];
+                    b = rps[row - n_lo + 1];
+                }
+                float r[MX];
+#pragma unroll
+                for (int m = 0; m < MX; ++m) r[m] = 0.f;
+#pragma unroll 1
+                for (int e = a + rl; e < b; e += 16) entry(e, r);
+#pragma unroll
+                for (int off = 8; off > 0; off >>= 1)
+#pragma unroll
+                    for (int m = 0; m < MX; ++m) r[m] += __shfl_xor_sync(0xffffffffu, r[m], off);
+                if (rl < M) {
+                    float v = r[0];
+#pragma unroll
+                    for (int m = 1; m < MX; ++m)
+                        if (m == rl) v = r[m];
+                    res[(k * M + rl) * 16 + hw] = b > a ? rsf[row - n_lo] * v : 0.f;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // ------------------------------------------------ reduction-add and store
+    for (int o = threadIdx.x; o < nt * M * 16; o += kThreads) {
+        const int k = o / (M * 16), rem = o - k * M * 16, m = rem >> 4, rr = rem & 15;
+        const int n = (t0 + k) * 16 + rr;
+        float y = resid ? res[(k * M + m) * 16 + rr] : 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) y += red[((k * kWarps + w) * M + m) * 16 + rr];
+        if (n < N) {
+            if (p.Yf)
+                p.Yf[static_cast<size_t>(m) * N + n] = y;
+            else
+                p.Y[static_cast<size_t>(m) * N + n] = __float2bfloat16_rn(y);
+        }
+    }
+    cp_async_wait_all();
+}
+
+template <int MX>
+void *kernel_for(int nt) {
+    switch (nt) {
+        case 1: return reinterpret_cast<void *>(decode_stream_kernel<MX, 1>);
+        case 2: return reinterpret_cast<void *>(decode_stream_kernel<MX, 2>);
+        case 3: return reinterpret_cast<void *>(decode_stream_kernel<MX, 3>);
+        case 4: return reinterpret_cast<void *>(decode_stream_kernel<MX, 4>);
+        case 5: return reinterpret_cast<void *>(decode_stream_kernel<MX, 5>);
+        case 6: return reinterpret_cast<void *>(decode_stream_kernel<MX, 6>);
+        case 7: return reinterpret_cast<void *>(decode_stream_kernel<MX, 7>);
+        default: return reinterpret_cast<void *>(decode_stream_kernel<MX, 8>);
+    }
+}
+
+}  // namespace
+
+mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y,
+                               cudaStream_t stream, float *partial, const L2Prefetch &pf) {
+    const DeviceWeight &d = weight_device(w);
+    if (M < 1 || M > 8) return MQ_ERR_UNSUPPORTED;
+    const int64_t ntile = (d.N + 15) / 16;
+    // one CTA per SM with NT = ceil(tiles / SMs) tiles each, or more CTAs of
+    // kTMax tiles for layers taller than kTMax tiles per SM
+    int64_t grid = std::min<int64_t>(ntile, sm_count());
+    if ((ntile + grid - 1) / grid > kTMax) grid = (ntile + kTMax - 1) / kTMax;
+    const int nt = static_cast<int>((ntile + grid - 1) / grid);
+    const bool with_residual = partial == nullptr && d.nnz > 0;
+    const int64_t span = with_residual ? max_span_nnz(w, ntile, static_cast<int>(grid)) : 0;
+    // a CTA's CSR slice too long for its shared-memory budget (a dense or
+    // block-allocated residual): the register kernel takes the call
+    if (span * 5 / 2 + 96 > kCsrBudget) return MQ_ERR_UNSUPPORTED;
+    StreamParams p;
+    p.qweight = d.qweight;
+    p.sz = d.sz;
+    p.X = static_cast<const __nv_bfloat16 *>(X);
+    p.Y = static_cast<__nv_bfloat16 *>(Y);
+    p.Yf = partial;
+    p.row_ptr = d.row_ptr;
+    p.col = d.col;
+    p.val = d.val;
+    p.rscale = d.rscale;
+    p.M = M;
+    p.N = static_cast<int>(d.N);
+    p.K = static_cast<int>(d.K);
+    p.G = static_cast<int>(d.G);
+    p.Gp = static_cast<int>(d.Gp);
+    p.ntile = static_cast<int>(ntile);
+    p.csr_cap = with_residual ? static_cast<int>(std::max<int64_t>(span, 1)) : 0;
+    p.bias = 0x43004300u;
+    p.pf = pf;
+    const StreamLayout L(M, p.K, p.Gp, p.csr_cap, nt);
+    if (L.total > kMaxSmem) return MQ_ERR_UNSUPPORTED;
+    void *kern = M == 1 ? kernel_for<1>(nt) : kernel_for<8>(nt);
+    static bool configured[64][2][kTMax + 1] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
+    if (dev >= 0 && dev < 64 && !configured[dev][M > 1][nt]) {
+        // the largest shared-memory carveout for every decode kernel, so that
+        // consecutive launches of different layers can share an SM without
+        // waiting for it to drain and be reconfigured
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+            return fail(MQ_ERR_CUDA, "cudaFuncSetAttribute failed for the streaming decode kernel");
+        configured[dev][M > 1][nt] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(L.total);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    void *args[] = {&p};
+    const cudaError_t e = cudaLaunchKernelExC(&cfg, kern, args);
+    if (e != cudaSuccess)
+        return fail(MQ_ERR_CUDA, std::string("streaming decode launch: ") + cudaGetErrorString(e));
+    return MQ_OK;
+}
+
+}  // namespace mq

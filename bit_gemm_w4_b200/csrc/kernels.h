@@ -52,6 +52,11 @@ struct DeviceWeight {
 // tile height; the decode kernels size their shared-memory CSR slice with it).
 int64_t max_tile_nnz(const mq_weight *w, int bn);
 
+// Largest residual entry count over `parts` contiguous runs of 16-row tiles,
+// run b holding tiles [ntile * b / parts, ntile * (b + 1) / parts) (cached
+// per part count; the streaming decode kernel stages a run's CSR slice).
+int64_t max_span_nnz(const mq_weight *w, int64_t ntile, int parts);
+
 // Tensor maps of the prefill kernel (built once per handle).
 struct PrefillMaps {
     CUtensorMap w;  // qweight, box [128 rows][pw words]; 128-byte swizzle when pw = 32
@@ -84,6 +89,15 @@ struct L2Prefetch {
 // (the unfused path's first half); else Y (bf16) gets the fused result.
 mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t stream,
                         float *partial = nullptr, const L2Prefetch &pf = L2Prefetch());
+
+// Streaming decode kernel (decode_stream.cu) for M <= 8: persistent, one
+// CTA per SM over contiguous 16-row tiles, a per-thread cp.async prefetch
+// ring. `partial` and `pf` as for launch_decode. Returns
+// MQ_ERR_UNSUPPORTED (without setting an error message) when X does not fit
+// its shared memory; the caller then takes the register kernel.
+mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y,
+                               cudaStream_t stream, float *partial = nullptr,
+                               const L2Prefetch &pf = L2Prefetch());
 
 // Wide decode kernel (decode_wide.cu) for 8 < M <= 16; `partial` as for
 // decode. Returns MQ_ERR_UNSUPPORTED (without setting an error message) when
