@@ -251,6 +251,27 @@ __device__ __forceinline__ uint32_t nib_pair_bias128(uint32_t w) {
     return (w & 0x000F000Fu) | 0x43004300u;
 }
 
+// The bias words of the code conversions, bf16x2 (128, 128) and the int8
+// sign-bias bytes. Kernels take them as launch parameters: held in a
+// register, (w & mask) | bias is one LOP3, where a second 32-bit immediate
+// would cost a second one.
+constexpr uint32_t kBiasBf16 = 0x43004300u;
+constexpr uint32_t kBiasI8 = 0x80808080u;
+
+template <uint32_t kMask>
+__device__ __forceinline__ uint32_t mask_or(uint32_t w, uint32_t bias) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(kMask), "r"(bias));
+    return d;
+}
+
+// Four int8 bytes q - z from the low nibble of each byte of w, with the
+// sign-bias word in a register (kBiasI8): the same arithmetic as
+// codes_minus_zero in two LOP3s and one add.
+__device__ __forceinline__ uint32_t codes_minus_zero_r(uint32_t w, uint32_t zz4, uint32_t bias8) {
+    return (mask_or<0x0F0F0F0Fu>(w, bias8) - zz4) ^ bias8;
+}
+
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));

@@ -60,6 +60,7 @@ struct DecodeParams {
     const uint8_t *val;
     const uint16_t *rscale;
     int M, N, K, G, Gp;
+    uint32_t bias;  // kBiasBf16, or kBiasI8 for int8 codes (held in a register)
     int csr_cap;  // residual entries staged in shared memory (0: read from global)
     int with_residual;
     L2Prefetch pf;  // the next layer's weight, brought into L2 meanwhile
@@ -110,6 +111,7 @@ __global__ void __launch_bounds__(Cfg<MX, RT, S, BG, CS>::THREADS)
     using C = Cfg<MX, RT, S, BG, CS>;
     constexpr int NT = C::NT, BN = C::BN;
     extern __shared__ __align__(16) uint8_t smem[];
+    const uint32_t bias = p.bias;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -289,10 +291,10 @@ __global__ void __launch_bounds__(Cfg<MX, RT, S, BG, CS>::THREADS)
                 const uint32_t a_lo = wr0[ks >> 1] >> (8 * (ks & 1));
                 const uint32_t b_lo = wr1[ks >> 1] >> (8 * (ks & 1));
                 uint32_t a[4];
-                a[0] = bf16x2_sub(nib_pair_bias128(a_lo), zz0);
-                a[1] = bf16x2_sub(nib_pair_bias128(b_lo), zz1);
-                a[2] = bf16x2_sub(nib_pair_bias128(a_lo >> 4), zz0);
-                a[3] = bf16x2_sub(nib_pair_bias128(b_lo >> 4), zz1);
+                a[0] = bf16x2_sub(mask_or<0x000F000Fu>(a_lo, bias), zz0);
+                a[1] = bf16x2_sub(mask_or<0x000F000Fu>(b_lo, bias), zz1);
+                a[2] = bf16x2_sub(mask_or<0x000F000Fu>(a_lo >> 4, bias), zz0);
+                a[3] = bf16x2_sub(mask_or<0x000F000Fu>(b_lo >> 4, bias), zz1);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
                     mma_bf16_16816(c[nt], a, xb[nt][2 * ks], xb[nt][2 * ks + 1], c[nt]);
@@ -380,6 +382,7 @@ mq_status run(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t st
     p.K = static_cast<int>(d.K);
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
+    p.bias = kBiasBf16;
     p.with_residual = with_residual ? 1 : 0;
     p.pf = pf;
     // The tile's CSR slice is staged in shared memory while that keeps two
@@ -396,8 +399,12 @@ mq_status run(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t st
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
     if (dev >= 0 && dev < 64 && !configured[dev]) {
+        // the largest shared-memory carveout, as for every decode kernel, so
+        // that consecutive launches of different layers can share an SM
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-            cudaSuccess)
+                cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return fail(MQ_ERR_CUDA, "cudaFuncSetAttribute failed for the decode kernel");
         configured[dev] = true;
     }

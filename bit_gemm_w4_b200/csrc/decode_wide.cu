@@ -89,6 +89,7 @@ struct WideParams {
     const uint16_t *went;
     const uint16_t *rscale;
     int M, N, K, G, Gp;
+    uint32_t bias;  // kBiasBf16, or kBiasI8 for int8 codes (held in a register)
     int S;           // stages over all of K
     int ent_bytes;   // residual entry bytes of one slot; 0 = no residual
     int x_off;       // X's offset in a slot (kEntOff + ent_bytes)
@@ -128,6 +129,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     decode_wide_kernel(const __grid_constant__ WideParams p) {
     constexpr int XRS = x_row_stride<A4>();
     extern __shared__ __align__(128) uint8_t smem[];
+    const uint32_t bias = p.bias;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int M = p.M, N = p.N, K = p.K, G = p.G;
@@ -298,10 +300,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     uint32_t a[4];
-                    a[0] = codes_minus_zero(wr0[ks] & 0x0F0F0F0Fu, zz0);
-                    a[1] = codes_minus_zero(wr1[ks] & 0x0F0F0F0Fu, zz1);
-                    a[2] = codes_minus_zero((wr0[ks] >> 4) & 0x0F0F0F0Fu, zz0);
-                    a[3] = codes_minus_zero((wr1[ks] >> 4) & 0x0F0F0F0Fu, zz1);
+                    a[0] = codes_minus_zero_r(wr0[ks], zz0, bias);
+                    a[1] = codes_minus_zero_r(wr1[ks], zz1, bias);
+                    a[2] = codes_minus_zero_r(wr0[ks] >> 4, zz0, bias);
+                    a[3] = codes_minus_zero_r(wr1[ks] >> 4, zz1, bias);
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) mma_s8_16832(d[nt], a, xb[nt][2 * ks], xb[nt][2 * ks + 1]);
                 }
@@ -325,10 +327,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const uint32_t a_lo = wr0[ks >> 1] >> (8 * (ks & 1));
                     const uint32_t b_lo = wr1[ks >> 1] >> (8 * (ks & 1));
                     uint32_t a[4];
-                    a[0] = bf16x2_sub(nib_pair_bias128(a_lo), zz0);
-                    a[1] = bf16x2_sub(nib_pair_bias128(b_lo), zz1);
-                    a[2] = bf16x2_sub(nib_pair_bias128(a_lo >> 4), zz0);
-                    a[3] = bf16x2_sub(nib_pair_bias128(b_lo >> 4), zz1);
+                    a[0] = bf16x2_sub(mask_or<0x000F000Fu>(a_lo, bias), zz0);
+                    a[1] = bf16x2_sub(mask_or<0x000F000Fu>(b_lo, bias), zz1);
+                    a[2] = bf16x2_sub(mask_or<0x000F000Fu>(a_lo >> 4, bias), zz0);
+                    a[3] = bf16x2_sub(mask_or<0x000F000Fu>(b_lo >> 4, bias), zz1);
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt)
                         mma_bf16_16816(c[nt], a, xb[nt][2 * ks], xb[nt][2 * ks + 1], c[nt]);
@@ -476,6 +478,7 @@ mq_status launch(WideParams &p, const DeviceWeight &d, int M, bool with_res, boo
     p.K = static_cast<int>(d.K);
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
+    p.bias = A4 ? kBiasI8 : kBiasBf16;
     p.S = static_cast<int>((d.K + kKC - 1) / kKC);
     const int64_t blocks = (d.N + kBN - 1) / kBN;
     if (blocks < sm_count() && !force) return MQ_ERR_UNSUPPORTED;  // the narrow kernels serve small layers

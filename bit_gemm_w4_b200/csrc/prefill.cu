@@ -102,6 +102,7 @@ struct PrefillParams {
     int pw;       // words per row of a packed-code box (32, or 16 when K = 128)
     int m_tiles;  // token tiles; tile t covers rows (t / m_tiles) and tokens (t % m_tiles)
     int tiles;
+    uint32_t bias;  // kBiasBf16, or kBiasI8 for the W4A4 form (held in a register)
 };
 
 struct SmemLayout {
@@ -561,6 +562,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     ++pc;
                 }
                 uint32_t codes[32];
+                const uint32_t bias = p.bias;
                 if constexpr (A4) {
                     // a word's low nibbles are its columns in positions 0-3 of the
                     // chunk's code order, the high nibbles positions 4-7: one
@@ -568,8 +570,8 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     const uint32_t zz = z * 0x01010101u;
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        codes[2 * c] = codes_minus_zero(words[c] & 0x0F0F0F0Fu, zz);
-                        codes[2 * c + 1] = codes_minus_zero((words[c] >> 4) & 0x0F0F0F0Fu, zz);
+                        codes[2 * c] = codes_minus_zero_r(words[c], zz, bias);
+                        codes[2 * c + 1] = codes_minus_zero_r(words[c] >> 4, zz, bias);
                     }
                 } else {
                     const uint32_t zz = (0x4300u | z) * 0x00010001u;  // bf16x2 (128 + z)
@@ -578,7 +580,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                         // pair j of word c holds columns (8c + 2j, 8c + 2j + 1)
 #pragma unroll
                         for (int jj = 0; jj < 4; ++jj)
-                            codes[4 * c + jj] = bf16x2_sub(nib_pair_bias128(words[c] >> (4 * jj)), zz);
+                            codes[4 * c + jj] = bf16x2_sub(mask_or<0x000F000Fu>(words[c] >> (4 * jj), bias), zz);
                     }
                 }
                 tmem_st32(tl + a * A_SLOT, codes);
@@ -760,6 +762,7 @@ mq_status launch_prefill_impl(const mq_weight *w, const void *X, const float *xs
     p.K = static_cast<int>(d.K);
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
+    p.bias = A4 ? kBiasI8 : kBiasBf16;
     p.m_tiles = static_cast<int>((M + BM - 1) / BM);
     const int64_t tiles = ((d.N + BN - 1) / BN) * static_cast<int64_t>(p.m_tiles);
     if (tiles > (int64_t(1) << 30)) return fail(MQ_ERR_UNSUPPORTED, "prefill kernel: too many tiles");

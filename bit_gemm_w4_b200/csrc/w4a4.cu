@@ -106,6 +106,7 @@ struct A4Params {
     const uint8_t *val;
     const uint16_t *rscale;
     int M, N, K, G, Gp;
+    uint32_t bias;  // kBiasBf16, or kBiasI8 for int8 codes (held in a register)
     int csr_cap;  // residual entries staged in shared memory (0: read from global)
 };
 
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(A4Cfg<MX, RT, S, BG, CS>::THREADS)
     using C = A4Cfg<MX, RT, S, BG, CS>;
     constexpr int NT = C::NT, BN = C::BN;
     extern __shared__ __align__(16) uint8_t smem[];
+    const uint32_t bias = p.bias;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -326,10 +328,10 @@ __global__ void __launch_bounds__(A4Cfg<MX, RT, S, BG, CS>::THREADS)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 uint32_t a[4];
-                a[0] = codes_minus_zero(wr0[ks] & 0x0F0F0F0Fu, zz0);
-                a[1] = codes_minus_zero(wr1[ks] & 0x0F0F0F0Fu, zz1);
-                a[2] = codes_minus_zero((wr0[ks] >> 4) & 0x0F0F0F0Fu, zz0);
-                a[3] = codes_minus_zero((wr1[ks] >> 4) & 0x0F0F0F0Fu, zz1);
+                a[0] = codes_minus_zero_r(wr0[ks], zz0, bias);
+                a[1] = codes_minus_zero_r(wr1[ks], zz1, bias);
+                a[2] = codes_minus_zero_r(wr0[ks] >> 4, zz0, bias);
+                a[3] = codes_minus_zero_r(wr1[ks] >> 4, zz1, bias);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) mma_s8_16832(d[nt], a, xb[nt][2 * ks], xb[nt][2 * ks + 1]);
             }
@@ -436,6 +438,7 @@ mq_status run_a4(const mq_weight *w, const int8_t *codes, const float *xscale, i
     p.K = static_cast<int>(d.K);
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
+    p.bias = kBiasI8;
     // stage the tile's CSR slice while that keeps two CTAs per SM
     p.csr_cap = static_cast<int>(std::min<int64_t>(tile_nnz, int64_t(1) << 24));
     if (A4Layout(M, p.G, CS, S, MX, C::BN, p.csr_cap).total > 100 * 1024) p.csr_cap = 0;
@@ -447,8 +450,12 @@ mq_status run_a4(const mq_weight *w, const int8_t *codes, const float *xscale, i
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
     if (dev >= 0 && dev < 64 && !configured[dev]) {
+        // the largest shared-memory carveout, as for every decode kernel, so
+        // that consecutive launches of different layers can share an SM
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-            cudaSuccess)
+                cudaSuccess ||
+            cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return fail(MQ_ERR_CUDA, "cudaFuncSetAttribute failed for the W4A4 decode kernel");
         configured[dev] = true;
     }
