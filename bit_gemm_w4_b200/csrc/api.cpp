@@ -294,8 +294,7 @@ const PrefillMaps *prefill_maps(const mq_weight *w) {
     if (!m) return nullptr;
     const DeviceWeight &d = w->d;
     m->pw = static_cast<int>(std::min<int64_t>(32, d.K / 8));
-    if (d.Gp > 256 ||
-        !encode_2d(&m->w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, d.qweight, d.K / 8, d.N, m->pw, 128,
+    if (!encode_2d(&m->w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, d.qweight, d.K / 8, d.N, m->pw, 128,
                    m->pw == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE)) {
         delete m;
         fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill maps");

@@ -14,8 +14,11 @@
 // library's code is loaded holds its kNoallocMaxOutputs floats until the
 // process exits. Host code cannot use the variable's name as a device
 // address, so the first call on each device (with that device current)
-// looks the address up with cudaGetSymbolAddress and caches it; make that
-// first call before any stream capture. All calls on a device share the one
+// looks the address up with cudaGetSymbolAddress and caches it, keyed on the
+// device and its current CUDA context: a call under another context (after
+// cudaDeviceReset, or with a non-primary context current) looks the address
+// up again. Make the first call on a device, and the first under a new
+// context, before any stream capture. All calls on a device share the one
 // array and it keeps the last call's contents; nothing in it has to start at
 // zero, because the dense kernel writes all M*N partials before the
 // residual kernel reads them. Calls whose GPU work overlaps (other streams,
@@ -35,22 +38,48 @@ constexpr int64_t kNoallocMaxOutputs = MQ_UNFUSED_NOALLOC_MAX_OUTPUTS;
 static __device__ __align__(256) float g_unfused_scratch[kNoallocMaxOutputs];
 
 std::mutex g_scratch_mu;
-void *g_scratch_ptr[256] = {};
+struct ScratchEntry {
+    CUcontext ctx = nullptr;
+    void *ptr = nullptr;
+};
+ScratchEntry g_scratch[256];
 
-// Device address of g_unfused_scratch on `dev` (the current device).
+// The driver's cuCtxGetCurrent, reached through the runtime (the library
+// links the CUDA runtime only).
+CUresult current_context(CUcontext *ctx) {
+    using Fn = CUresult (*)(CUcontext *);
+    static Fn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<Fn>(p);
+    });
+    return fn ? fn(ctx) : CUDA_ERROR_NOT_FOUND;
+}
+
+// Device address of g_unfused_scratch on `dev` (the current device) in the
+// current context.
 mq_status scratch_address(int dev, float **out) {
     if (dev < 0 || dev >= 256) return fail(MQ_ERR_UNSUPPORTED, "device ordinal out of range");
+    CUcontext ctx = nullptr;
+    if (current_context(&ctx) != CUDA_SUCCESS || !ctx)
+        return fail(MQ_ERR_CUDA, "no current CUDA context for the built-in scratch");
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
+    ScratchEntry &e = g_scratch[dev];
+    if (!e.ptr || e.ctx != ctx) {
         void *p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_unfused_scratch);
-        if (e != cudaSuccess || !p)
+        const cudaError_t r = cudaGetSymbolAddress(&p, g_unfused_scratch);
+        if (r != cudaSuccess || !p)
             return fail(MQ_ERR_CUDA, std::string("cudaGetSymbolAddress for the built-in "
                                                  "scratch failed: ") +
-                                         cudaGetErrorString(e));
-        g_scratch_ptr[dev] = p;
+                                         cudaGetErrorString(r));
+        e.ctx = ctx;
+        e.ptr = p;
     }
-    *out = static_cast<float *>(g_scratch_ptr[dev]);
+    *out = static_cast<float *>(e.ptr);
     return MQ_OK;
 }
 

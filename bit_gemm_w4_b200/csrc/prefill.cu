@@ -735,7 +735,6 @@ template <bool A4>
 mq_status launch_prefill_impl(const mq_weight *w, const void *X, const float *xscale, int64_t M,
                               void *Y, cudaStream_t stream, float *partial) {
     const DeviceWeight &d = weight_device(w);
-    if (d.Gp > 256) return fail(MQ_ERR_UNSUPPORTED, "prefill kernel: K above 32768");
     if (M > (int64_t(1) << 23)) return fail(MQ_ERR_UNSUPPORTED, "prefill kernel: M above 2^23");
     if (A4 && d.K % 256) return fail(MQ_ERR_UNSUPPORTED, "W4A4 prefill kernel: K must be a multiple of 256");
     const PrefillMaps *pm = prefill_maps(w);

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libmosaicq.so")
 
 OK, INVALID_ARG, UNSUPPORTED, OUT_OF_MEMORY, CUDA, DEVICE_TIMEOUT = range(6)
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = range(3)
+UNFUSED_NOALLOC_MAX_OUTPUTS = 2 * 1024 * 1024  # MQ_UNFUSED_NOALLOC_MAX_OUTPUTS
 _PATHS = {"auto": PATH_AUTO, "decode": PATH_DECODE, "prefill": PATH_PREFILL}
 
 
@@ -67,6 +68,7 @@ def _load():
         "mq_linear_unfused_noalloc": ([vp, vp, i64, vp, vp], st),
         "mq_quantize_activations": ([vp, i64, i64, vp, vp, vp], st),
         "mq_selftest_bounded_wait": ([i64, ctypes.POINTER(ctypes.c_int32)], st),
+        "mq_read_probe": ([vp, i64, vp, vp], st),
         "mq_w4a4_workspace_bytes": ([vp, i64], i64),
         "mq_linear_w4a4": ([vp, vp, i64, vp, vp, ctypes.c_size_t, vp], st),
         "mq_free": ([vp], None),
@@ -194,6 +196,13 @@ def selftest_bounded_wait(limit_cycles: int = 1 << 20) -> list:
     out = (ctypes.c_int32 * 4)()
     _check(_lib.mq_selftest_bounded_wait(int(limit_cycles), out), "mq_selftest_bounded_wait")
     return list(out)
+
+
+def read_probe(buf_ptr: int, nbytes: int, sink_ptr: int, *, stream=None) -> None:
+    """One launch of the library's streaming-read probe (mq_read_probe) over
+    nbytes of device memory at buf_ptr; sink_ptr is a 4-byte device word."""
+    _check(_lib.mq_read_probe(ctypes.c_void_p(buf_ptr), int(nbytes), ctypes.c_void_p(sink_ptr),
+                              _stream(stream)), "mq_read_probe")
 
 
 def quantize_activations(X, *, stream=None):

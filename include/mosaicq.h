@@ -139,10 +139,13 @@ mq_status mq_pack(const float *W_host, int64_t N, int64_t K,
  * allocation. X and Y are bf16, row-major, device memory of the packing
  * device, 16-byte aligned; Y is overwritten and must not overlap X. The
  * handle is read-only here, so concurrent calls on different streams are
- * safe. M = 0 launches nothing.
+ * safe. M = 0 launches nothing. Every K that mq_pack accepts (up to 65536)
+ * is served at every M.
  * Errors: INVALID_ARG for a NULL handle, NULL X/Y with M > 0, M < 0,
- * misaligned X/Y or a current device other than the packing device; CUDA
- * when a launch fails. */
+ * misaligned X/Y or a current device other than the packing device;
+ * UNSUPPORTED for M above 2^23 (more than M = 16 runs the prefill kernel,
+ * whose token tiles are counted in 32 bits) or a device ordinal above 63;
+ * CUDA when a launch fails. */
 mq_status mq_linear(const mq_weight *w, const void *X_dev, int64_t M,
                     void *Y_dev, mq_stream stream);
 
@@ -192,7 +195,9 @@ mq_status mq_linear_unfused(const mq_weight *w, const void *X_dev, int64_t M,
  * loads the library until the process exits) and performs no allocation of
  * any kind. Results match mq_linear_unfused.
  * The first call on each device looks up the array's device address with
- * that device current; make it before any stream capture. All calls on a
+ * that device current, and looks it up again when called under another
+ * CUDA context of the device (after cudaDeviceReset, or with a non-primary
+ * context current); make such first calls before any stream capture. All calls on a
  * device share the array, which keeps the last call's contents (nothing in
  * it needs to start at zero); calls whose GPU work overlaps in time race.
  * Errors as mq_linear, plus INVALID_ARG when M*N exceeds
@@ -255,6 +260,21 @@ void mq_free(mq_weight *w);
  * is never hung: the stuck wait ends after its limit.
  * Errors: INVALID_ARG for NULL results or a limit outside (0, 2^31]; CUDA. */
 mq_status mq_selftest_bounded_wait(int64_t limit_cycles, int32_t *results);
+
+/* A measuring aid with no counterpart in the paper: one pure streaming read
+ * of `bytes` bytes at buf_dev (device memory, 16-byte aligned, bytes a
+ * positive multiple of 16), shaped for the attainable HBM read bandwidth: a
+ * persistent grid of two CTAs per SM over contiguous stretches, eight
+ * 16-byte streaming loads in flight per thread, programmatic dependent
+ * launch (the next launch is released at once; this one waits for its
+ * predecessor only before its last write). sink_dev (4 bytes, device) is
+ * written only on a data pattern that practically never occurs, so the
+ * loads cannot be dropped. Asynchronous on `stream`; the caller owns both
+ * buffers. A graph of these launches with a decode step's byte counts gives
+ * the read ceiling for that chain of launches.
+ * Errors: INVALID_ARG for NULL or misaligned pointers or a bad size; CUDA
+ * when the launch fails. */
+mq_status mq_read_probe(const void *buf_dev, int64_t bytes, void *sink_dev, mq_stream stream);
 
 /* Residual entries a pack with these options produces: N * k_n in row mode,
  * (selected blocks) * 1024 in block mode. */

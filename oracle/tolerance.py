@@ -3,15 +3,17 @@
 Test infrastructure (see oracle/__init__.py).
 
 Two bounds accept an output y against the fp64 value y64:
-  T1 normalized error  (|y - y64| - ulp(y64)) / (||x_m|| * ||w_hat_n||) <= 2e-3
+  T1 normalized error  (|y - y64| - ulp(y64) / 2) / (||x_m|| * ||w_hat_n||) <= 2e-3
   T2 relative error    |y - y64| / |y64| <= 1e-2 wherever |y64| > 1e-3
 
 Reading of T1: the outputs are bf16, whose unit roundoff is 2^-8 (3.9e-3)
 relative. Rounding even the exact y64 to bf16 can exceed 2e-3 * ||x|| * ||w||
 whenever |y64| is more than about half of ||x|| * ||w|| (x and the weight row
 nearly parallel), so the normalized bound is applied to the error in excess
-of one bf16 ulp at y64, the spacing of the output grid there. T2 needs no such
-allowance (1e-2 is above the bf16 roundoff).
+of half a bf16 ulp at y64: the most that rounding y64 to the nearest point of
+the output grid can add. T2 needs no such allowance (1e-2 is above the bf16
+roundoff). The report also gives t1_raw, the normalized error with no
+allowance.
 """
 
 from __future__ import annotations
@@ -39,7 +41,7 @@ def parity_report(Y, Y64: np.ndarray, X64: np.ndarray,
     diff = np.abs(Y - Y64)
     xn = np.linalg.norm(X64, axis=1)[:, None]
     denom = xn * np.asarray(w_rows_norm, np.float64)[None, :]
-    excess = np.maximum(diff - bf16_ulp(Y64), 0.0)
+    excess = np.maximum(diff - 0.5 * bf16_ulp(Y64), 0.0)
     t1 = np.where(denom > 0, excess / np.where(denom > 0, denom, 1.0), excess)
     t1_raw = np.where(denom > 0, diff / np.where(denom > 0, denom, 1.0), diff)
     big = np.abs(Y64) > T2_FLOOR

@@ -347,6 +347,18 @@ def test_longest_k_decode(mq, cuda, M):
     assert r["ok"], r
 
 
+@pytest.mark.parametrize("M", [17, 40])
+def test_longest_k_prefill(mq, cuda, M):
+    # K = 65536 at more than 16 tokens: the prefill kernel reads 512 scale
+    # words per row (beyond the 256 of its first design)
+    N, K = 160, 65536
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=96)
+    X = synth.activations(M, K, seed=97, channels=4, mult=20.0)
+    w, Y = _run(mq, W, X, 0.002)
+    r = oracle_check(Y, X, oracle.decompose(W, 0.002))
+    assert r["ok"], r
+
+
 def test_bounded_wait_gives_up(mq, cuda):
     # a wait on a barrier phase nobody completes ends after its limit with
     # its code in the error word, and the wait after it returns at once

@@ -73,3 +73,11 @@ def test_injected_allocation_failure(mq, monkeypatch):
         mq.Weight.pack(W, 0.02, stream=0)      # the default stream: no torch CUDA call
     assert e.value.status == mq.OUT_OF_MEMORY
     assert b"MQ_FAULT_ALLOC" in mq.lib().mq_last_error()
+
+
+def test_noalloc_capacity_constant_matches_header():
+    import re
+    from bit_gemm_w4_b200 import mosaicq as mq
+    hdr = open(os.path.join(ROOT, "include", "mosaicq.h")).read()
+    m = re.search(r"#define MQ_UNFUSED_NOALLOC_MAX_OUTPUTS \(([^)]*)\)", hdr)
+    assert m and eval(m.group(1), {}) == mq.UNFUSED_NOALLOC_MAX_OUTPUTS

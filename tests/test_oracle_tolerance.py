@@ -34,3 +34,20 @@ def test_exact_rounding_passes_and_real_errors_fail():
     i = np.argmax(np.abs(Y64[2]) > 0.5)
     bad[2, i] *= 1.05                                       # 5 % relative error
     assert not parity_report(bad, Y64, X, wn)["ok"]
+
+
+def test_t1_allows_half_an_ulp_not_one():
+    # a weight row exactly parallel to x, scaled so that y64 sits just above
+    # a power of two: there |y64| ~ ||x|| ||w|| and one bf16 ulp is |y64|/128
+    x = np.ones((1, 128))
+    w = np.ones((1, 128)) * (1.01 / 128)
+    Y64 = x @ w.T                                    # 1.01
+    wn = np.linalg.norm(w, axis=1)
+    Yb = torch.from_numpy(Y64).to(torch.bfloat16).double().numpy()
+    r = parity_report(Yb, Y64, x, wn)
+    assert r["ok"] and r["t1"] == 0.0                # correct rounding passes
+    assert r["t1_raw"] > 2e-3                        # which alone would exceed the bound
+    u = bf16_ulp(Y64)
+    assert parity_report(Y64 + 0.5 * u, Y64, x, wn)["t1"] == 0.0    # half an ulp: free
+    assert not parity_report(Y64 + u, Y64, x, wn)["ok"]            # one full ulp off fails
+    assert not parity_report(Y64 - u, Y64, x, wn)["ok"]
