@@ -9,7 +9,8 @@ the MosaicQuant pages:
     equation W_hat ~= Q(W_hat) + R; both parts 4-bit), with the residual
     allocated per row or per block ("Methodology" 2, the Hessian-guided
     delta score).
-  * pack.py      - the device byte layout of that decomposition, and unpack.
+  * pack.py      - the device byte layout of that decomposition, and unpack;
+                   the block-tile layout of a block-allocated residual.
   * linear.py    - the product Y = X * W_hat^T, W_hat = deq(Q) + R, as dense
     base plus a CSR loop (the "reduction-add" of ZipperEngine's pipeline) and
     as a brute-force triple loop.
@@ -29,13 +30,14 @@ from .decompose import (Decomposition, decompose, from_arrays, fp16_rne,
                         residual_count, quantize_base, select_residual,
                         quantize_residual, decompose_blocks, block_scores,
                         select_blocks, blocks_selected)
-from .pack import pack, unpack
+from .pack import pack, unpack, block_structure, pack_blocks, unpack_blocks
 from .linear import dequant_base, w_hat, linear, linear_brute
 from .tolerance import parity_report
 
 __all__ = [
     "Decomposition", "decompose", "from_arrays", "fp16_rne", "residual_count",
     "quantize_base", "select_residual", "quantize_residual", "pack", "unpack",
+    "block_structure", "pack_blocks", "unpack_blocks",
     "dequant_base", "w_hat", "linear", "linear_brute", "parity_report",
     "decompose_blocks", "block_scores", "select_blocks", "blocks_selected",
 ]

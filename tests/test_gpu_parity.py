@@ -347,6 +347,23 @@ def test_longest_k_decode(mq, cuda, M):
     assert r["ok"], r
 
 
+@pytest.mark.parametrize("M,K,rho", [(9, 2176, 0.01), (16, 2176, 0.04), (16, 1024, 0.01), (12, 640, 0.0)])
+def test_tall_layer_decode(mq, cuda, M, K, rho):
+    # 9-16 tokens on a layer tall enough for the wide kernel (19000 rows: the
+    # last 16-row tile ragged); K = 2176 ends in a half stage
+    N = 19000
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=M + K)
+    X = synth.activations(M, K, seed=31 + M, channels=4, mult=20.0)
+    w, Y = _run(mq, W, X, rho)
+    d = oracle.decompose(W, rho)
+    r = oracle_check(Y, X, d)
+    assert r["ok"], r
+    Yu = w.linear_unfused(X.cuda())      # the split execution's dense half without residual
+    torch.cuda.synchronize()
+    ru = oracle_check(Yu, X, d)
+    assert ru["ok"], ru
+
+
 @pytest.mark.parametrize("M", [17, 40])
 def test_longest_k_prefill(mq, cuda, M):
     # K = 65536 at more than 16 tokens: the prefill kernel reads 512 scale
