@@ -30,6 +30,8 @@ struct mq_weight {
     mutable std::mutex maps_mu;
     mutable std::vector<std::pair<int, int64_t>> tile_nnz;  // (tile height, max entries)
     mutable std::vector<std::pair<int, int64_t>> span_nnz;  // (CTA count, max entries)
+    mutable std::vector<std::pair<int, int64_t>> span_blk;  // (CTA count, max blocks)
+    std::vector<int32_t> host_blk_ptr;                      // block tiles: offsets per block-row
     mutable mq::PrefillMaps *pmaps = nullptr;
     ~mq_weight() { delete pmaps; }
 };
@@ -209,6 +211,16 @@ mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **o
         if (!st) st = upload(w, &woff, hwoff.data(), hwoff.size(), 0, stream);
         if (!st) st = upload(w, &went, hwent.data(), hwent.size(), 64, stream);
     }
+    int32_t *bptr = nullptr;
+    uint16_t *bcol = nullptr;
+    uint32_t *bq = nullptr, *bmap = nullptr;
+    HostBlocks hb;
+    if (!st && block_tiles_host(hp, hb)) {
+        st = upload(w, &bptr, hb.ptr.data(), hb.ptr.size(), 0, stream);
+        if (!st) st = upload(w, &bcol, hb.col.data(), hb.col.size(), 64, stream);
+        if (!st) st = upload(w, &bq, hb.q.data(), hb.q.size(), 0, stream);
+        if (!st) st = upload(w, &bmap, hb.map.data(), hb.map.size(), 0, stream);
+    }
     if (!st) st = upload(w, &err, &zero, 1, 0, stream);
     if (!st) {
         e = cudaStreamSynchronize(stream);
@@ -230,6 +242,13 @@ mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **o
     d.wide_off = woff;
     d.wide_ent = went;
     d.wide_max = wide_max;
+    d.blk_ptr = bptr;
+    d.blk_col = bcol;
+    d.blk_q = bq;
+    d.blk_map = bmap;
+    d.nblk = bq ? hb.nblk : 0;
+    d.blk_words = bq ? hb.map_words : 0;
+    if (bq) w->host_blk_ptr = hb.ptr;
     d.err = err;
     w->host_row_ptr = hp.row_ptr;
     for (int64_t n = 0; n < hp.N; ++n)
@@ -284,6 +303,22 @@ int64_t max_span_nnz(const mq_weight *w, int64_t ntile, int parts) {
         mx = std::max<int64_t>(mx, w->host_row_ptr[r1] - w->host_row_ptr[r0]);
     }
     w->span_nnz.emplace_back(parts, mx);
+    return mx;
+}
+
+int64_t max_span_blocks(const mq_weight *w, int64_t ntile, int parts) {
+    if (w->host_blk_ptr.empty()) return 0;
+    std::lock_guard<std::mutex> lock(w->maps_mu);
+    for (const auto &e : w->span_blk)
+        if (e.first == parts) return e.second;
+    int64_t mx = 0;
+    const int64_t nbr = static_cast<int64_t>(w->host_blk_ptr.size()) - 1;
+    for (int64_t b = 0; b < parts; ++b) {
+        const int64_t t0 = std::min<int64_t>(nbr, ntile * b / parts);
+        const int64_t t1 = std::min<int64_t>(nbr, ntile * (b + 1) / parts);
+        mx = std::max<int64_t>(mx, w->host_blk_ptr[t1] - w->host_blk_ptr[t0]);
+    }
+    w->span_blk.emplace_back(parts, mx);
     return mx;
 }
 
@@ -518,6 +553,57 @@ mq_status mq_export(const mq_weight *w, mq_host_packed *out) {
     cp(out->rscale, d.rscale, size_t(d.N) * 2);
     if (prev != w->device) cudaSetDevice(prev);
     if (e != cudaSuccess) return cuda_fail(e, "mq_export");
+    return MQ_OK;
+}
+
+namespace {
+mq_status copy_blocks_out(const HostBlocks &b, int32_t *blk_ptr, uint16_t *blk_col, uint32_t *blk_q,
+                          int64_t *nblk) {
+    *nblk = b.nblk;
+    if (!blk_ptr) return MQ_OK;
+    if (!blk_col || !blk_q) return fail(MQ_ERR_INVALID_ARG, "an output buffer is NULL");
+    std::memcpy(blk_ptr, b.ptr.data(), b.ptr.size() * 4);
+    std::memcpy(blk_col, b.col.data(), b.col.size() * 2);
+    std::memcpy(blk_q, b.q.data(), b.q.size() * 4);
+    return MQ_OK;
+}
+}  // namespace
+
+mq_status mq_block_tiles_host(const mq_decomp *d, int32_t *blk_ptr, uint16_t *blk_col,
+                              uint32_t *blk_q, int64_t *nblk) {
+    if (!d || !nblk) return fail(MQ_ERR_INVALID_ARG, "NULL pointer");
+    if (mq_status st = validate_decomp(d)) return st;
+    HostPacked p;
+    pack_host(*d, p);
+    HostBlocks b;
+    if (!block_tiles_host(p, b)) {
+        *nblk = 0;
+        return fail(MQ_ERR_UNSUPPORTED, "the residual is not made of whole 16 x 64 blocks");
+    }
+    return copy_blocks_out(b, blk_ptr, blk_col, blk_q, nblk);
+}
+
+mq_status mq_export_blocks(const mq_weight *w, int32_t *blk_ptr, uint16_t *blk_col, uint32_t *blk_q,
+                           int64_t *nblk) {
+    if (!w || !nblk) return fail(MQ_ERR_INVALID_ARG, "NULL pointer");
+    const DeviceWeight &d = w->d;
+    if (!d.blk_q) {
+        *nblk = 0;
+        return fail(MQ_ERR_UNSUPPORTED, "the weight has no block tiles");
+    }
+    *nblk = d.nblk;
+    if (!blk_ptr) return MQ_OK;
+    if (!blk_col || !blk_q) return fail(MQ_ERR_INVALID_ARG, "an output buffer is NULL");
+    int prev = -1;
+    if (cudaGetDevice(&prev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
+    if (prev != w->device && cudaSetDevice(w->device) != cudaSuccess)
+        return fail(MQ_ERR_CUDA, "cudaSetDevice failed");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(blk_ptr, d.blk_ptr, size_t(d.N / 16 + 1) * 4, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && d.nblk) e = cudaMemcpy(blk_col, d.blk_col, size_t(d.nblk) * 2, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && d.nblk) e = cudaMemcpy(blk_q, d.blk_q, size_t(d.nblk) * 512, cudaMemcpyDeviceToHost);
+    if (prev != w->device) cudaSetDevice(prev);
+    if (e != cudaSuccess) return cuda_fail(e, "mq_export_blocks");
     return MQ_OK;
 }
 

@@ -63,7 +63,8 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTMax = 8;     // most tiles per CTA (one accumulator set each)
 constexpr int kMaxSmem = 200 * 1024;
-constexpr int kCsrBudget = 24 * 1024;  // shared memory for a CTA's CSR slice
+constexpr int kCsrBudget = 24 * 1024;    // shared memory for a CTA's CSR slice
+constexpr int kBlockBudget = 48 * 1024;  // shared memory for a CTA's block tiles
 
 // Groups of prefetch ahead for NT tiles per CTA: eight to ten items per
 // thread (64-80 KB per CTA in flight), or one group for NT > 5.
@@ -83,7 +84,14 @@ struct StreamParams {
     const uint16_t *rscale;
     int M, N, K, G, Gp;
     int ntile;      // ceil(N / 16)
-    int csr_cap;    // most residual entries of a CTA's run; 0: no residual
+    int csr_cap;    // most residual entries of a CTA's run; 0: no CSR walk
+    // block tiles of a block-allocated residual (blk_cap > 0: the most blocks
+    // of a CTA's run; the residual then runs as tensor-core passes and the
+    // CSR is not read)
+    const int32_t *blk_ptr;
+    const uint32_t *blk_q;
+    const uint32_t *blk_map;
+    int blk_words, blk_cap;
     // 0x43004300 (bf16x2 128.0, 128.0), passed at run time so that it sits in
     // a register and each code pair costs one LOP3 (mask and OR)
     uint32_t bias;
@@ -96,8 +104,9 @@ __host__ __device__ inline int sz_stride(int Gp) { return ((Gp >> 2) & 1) ? Gp :
 
 // Shared-memory layout (bytes), identical on host and device.
 struct StreamLayout {
-    int ring, x, xrs, szs, red, res, rsf, rp, col, val, total;
-    __host__ __device__ StreamLayout(int M, int K, int Gp, int csr_cap, int nt) {
+    int ring, x, xrs, szs, red, res, rsf, rp, col, val, bq, bmap, bpre, total;
+    __host__ __device__ StreamLayout(int M, int K, int Gp, int csr_cap, int nt, int blk_cap = 0,
+                                     int blk_words = 0) {
         ring = 0;                                              // [D * NT][2][kThreads][16 B]
         x = ring + groups_ahead(nt) * nt * 2 * kThreads * 16;  // [M][xrs]
         xrs = K * 2 + 16;
@@ -108,7 +117,10 @@ struct StreamLayout {
         rp = rsf + nt * 16 * 4;                                // [NT * 16 + 1] i32
         col = rp + (csr_cap > 0 ? (nt * 16 + 1) * 4 + 15 : 0) / 16 * 16;
         val = col + (csr_cap > 0 ? csr_cap * 2 + 32 : 0);
-        total = val + (csr_cap > 0 ? csr_cap / 2 + 48 : 0);
+        bq = val + (csr_cap > 0 ? csr_cap / 2 + 48 : 0);                  // [blk_cap][512 B]
+        bmap = bq + blk_cap * 512;                                        // [NT][blk_words] bitmaps
+        bpre = bmap + (blk_cap > 0 ? nt * blk_words * 4 : 0);            // [NT][blk_words] block counts before each word
+        total = bpre + (blk_cap > 0 ? nt * blk_words * 4 : 0);
     }
 };
 
@@ -156,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int M = MX == 1 ? 1 : p.M, N = p.N, K = p.K, G = p.G;
-    const StreamLayout L(M, K, p.Gp, p.csr_cap, NT);
+    const StreamLayout L(M, K, p.Gp, p.csr_cap, NT, p.blk_cap, p.blk_words);
     const int SZS = sz_stride(p.Gp);
     const int t0 = static_cast<int>(static_cast<long long>(p.ntile) * blockIdx.x / gridDim.x);
     const int t1 = static_cast<int>(static_cast<long long>(p.ntile) * (blockIdx.x + 1) / gridDim.x);
@@ -164,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
     const bool full = nt == NT;  // only tile NT - 1 can be missing
     const int gpw = warp < G ? (G - warp + kWarps - 1) / kWarps : 0;  // groups of this warp
     const bool resid = p.csr_cap > 0;
+    const bool blocks = p.blk_cap > 0;
 
     // ------------------------------------------------ the weight stream
     // Row offsets (words) of this thread's rows g and g+8 in each tile, and
@@ -228,10 +241,29 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
         for (int i = threadIdx.x; i < nval16; i += kThreads)
             cp_async16(smem + L.val + 16 * i, p.val + val_base + 16 * i);
     }
+    int b_lo = 0;
+    if (blocks) {
+        // the run's block tiles (contiguous) and its block-rows' bitmaps
+        b_lo = p.blk_ptr[t0];
+        const int nb16 = (p.blk_ptr[t1] - b_lo) * 32;  // 16-byte pieces
+        for (int i = threadIdx.x; i < nb16; i += kThreads)
+            cp_async16(smem + L.bq + 16 * i, p.blk_q + static_cast<size_t>(b_lo) * 128 + 4 * i);
+        for (int i = threadIdx.x; i < nt * p.blk_words; i += kThreads)
+            cp_async4(smem + L.bmap + 4 * i, p.blk_map + static_cast<size_t>(t0) * p.blk_words + i);
+    }
     cp_async_commit();
-    if (resid)
+    if (resid || blocks)
         for (int i = threadIdx.x; i < n_hi - n_lo; i += kThreads)
             reinterpret_cast<float *>(smem + L.rsf)[i] = half_bits_to_f32(p.rscale[n_lo + i]);
+    if (blocks)
+        // each tile's blocks before each bitmap word, counted from the run's first block
+        for (int k = threadIdx.x; k < nt; k += kThreads) {
+            int c = p.blk_ptr[t0 + k] - b_lo;
+            for (int wd = 0; wd < p.blk_words; ++wd) {
+                reinterpret_cast<int *>(smem + L.bpre)[k * p.blk_words + wd] = c;
+                c += __popc(p.blk_map[static_cast<size_t>(t0 + k) * p.blk_words + wd]);
+            }
+        }
 
     // ------------------------------------------------ X
     pdl_wait();  // X may come from the previous kernel; Y may still be read by it
@@ -248,6 +280,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
 
     const uint8_t *xs = smem + L.x;
     const uint32_t *szs = reinterpret_cast<const uint32_t *>(smem + L.szs);
+    const uint32_t *bmapw = reinterpret_cast<const uint32_t *>(smem + L.bmap);
+    const int *bpre = reinterpret_cast<const int *>(smem + L.bpre);
+    const float *rsfs = reinterpret_cast<const float *>(smem + L.rsf);
     float *red = reinterpret_cast<float *>(smem + L.red);
     float *res = reinterpret_cast<float *>(smem + L.res);
 
@@ -279,6 +314,53 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
                         xb[4 * i + 3] = v.w;
                     }
                 }
+                // the residual blocks of tile k in group gi (column-blocks 2gi and
+                // 2gi + 1; lanes t = 0, 1 hold the first, t = 2, 3 the second):
+                // one more pass over the group's X fragment with offset-binary
+                // codes q_r + 8 (8, a zero residual, where a half has no
+                // block), scaled by each row's s_r
+                auto block_pass = [&](int k, int gi) {
+                    const int cb0 = 2 * gi;
+                    const uint32_t word = bmapw[k * p.blk_words + (cb0 >> 5)];
+                    const uint32_t two = (word >> (cb0 & 31)) & 3u;
+                    if (two == 0) return;
+                    const int lb0 = bpre[k * p.blk_words + (cb0 >> 5)] + __popc(word & ((1u << (cb0 & 31)) - 1u));
+                    const int h = t >> 1;
+                    const bool present = (two >> h) & 1u;
+                    const int lb = lb0 + (h ? static_cast<int>(two & 1u) : 0);
+                    uint4 ba = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u), bb = ba;
+                    if (present) {
+                        const uint8_t *bsrc = smem + L.bq + lb * 512 + (t & 1) * 16;
+                        ba = *reinterpret_cast<const uint4 *>(bsrc + g * 32);
+                        bb = *reinterpret_cast<const uint4 *>(bsrc + (g + 8) * 32);
+                    }
+                    const uint32_t bias = p.bias;
+                    const uint32_t zz = 0x43084308u;  // bf16x2 (136, 136): u - 8 = q_r exactly
+                    float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+                    const uint32_t wr0[4] = {ba.x, ba.y, ba.z, ba.w};
+                    const uint32_t wr1[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t a_lo = wr0[ks >> 1] >> (8 * (ks & 1));
+                        const uint32_t b_lo = wr1[ks >> 1] >> (8 * (ks & 1));
+                        uint32_t a[4];
+                        a[0] = bf16x2_sub(nib_pair(a_lo, bias), zz);
+                        a[1] = bf16x2_sub(nib_pair(b_lo, bias), zz);
+                        a[2] = bf16x2_sub(nib_pair(a_lo >> 4, bias), zz);
+                        a[3] = bf16x2_sub(nib_pair(b_lo >> 4, bias), zz);
+                        if (ks & 1)
+                            mma_pure(cb, a, xb[2 * ks], xb[2 * ks + 1]);
+                        else
+                            mma_pure(ca, a, xb[2 * ks], xb[2 * ks + 1]);
+                    }
+                    const float r0s = rsfs[k * 16 + g], r1s = rsfs[k * 16 + g + 8];
+                    acc[k][0] = fmaf(r0s, ca[0] + cb[0], acc[k][0]);
+                    acc[k][2] = fmaf(r1s, ca[2] + cb[2], acc[k][2]);
+                    if (MX > 1) {
+                        acc[k][1] = fmaf(r0s, ca[1] + cb[1], acc[k][1]);
+                        acc[k][3] = fmaf(r1s, ca[3] + cb[3], acc[k][3]);
+                    }
+                };
                 // one item: tile k of group gi, from ring slot d * NT + k
                 auto item = [&](int k) {
                     const uint8_t *src = ring + (d * NT + k) * (2 * kThreads * 16);
@@ -313,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
                         acc[k][1] = fmaf(s0, ca[1] + cb[1], acc[k][1]);
                         acc[k][3] = fmaf(s1, ca[3] + cb[3], acc[k][3]);
                     }
+                    if (blocks) block_pass(k, gi);
                 };
                 // items in pairs after one wait, so that the two interleave;
                 // each slot is refilled D groups ahead once its values are used
@@ -472,9 +555,13 @@ mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y
     if ((ntile + grid - 1) / grid > kTMax) grid = (ntile + kTMax - 1) / kTMax;
     const int nt = static_cast<int>((ntile + grid - 1) / grid);
     const bool with_residual = partial == nullptr && d.nnz > 0;
-    const int64_t span = with_residual ? max_span_nnz(w, ntile, static_cast<int>(grid)) : 0;
-    // a CTA's CSR slice too long for its shared-memory budget (a dense or
-    // block-allocated residual): the register kernel takes the call
+    // a block-allocated residual runs from its block tiles, a row residual
+    // from the CSR; a CTA's share too long for its shared-memory budget: the
+    // register kernel takes the call
+    const bool use_blocks = with_residual && d.blk_q != nullptr;
+    const int64_t bspan = use_blocks ? max_span_blocks(w, ntile, static_cast<int>(grid)) : 0;
+    if (bspan * 512 > kBlockBudget) return MQ_ERR_UNSUPPORTED;
+    const int64_t span = (with_residual && !use_blocks) ? max_span_nnz(w, ntile, static_cast<int>(grid)) : 0;
     if (span * 5 / 2 + 96 > kCsrBudget) return MQ_ERR_UNSUPPORTED;
     StreamParams p;
     p.qweight = d.qweight;
@@ -492,10 +579,15 @@ mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y
     p.G = static_cast<int>(d.G);
     p.Gp = static_cast<int>(d.Gp);
     p.ntile = static_cast<int>(ntile);
-    p.csr_cap = with_residual ? static_cast<int>(std::max<int64_t>(span, 1)) : 0;
+    p.csr_cap = (with_residual && !use_blocks) ? static_cast<int>(std::max<int64_t>(span, 1)) : 0;
+    p.blk_ptr = d.blk_ptr;
+    p.blk_q = d.blk_q;
+    p.blk_map = d.blk_map;
+    p.blk_words = static_cast<int>(d.blk_words);
+    p.blk_cap = use_blocks ? static_cast<int>(std::max<int64_t>(bspan, 1)) : 0;
     p.bias = 0x43004300u;
     p.pf = pf;
-    const StreamLayout L(M, p.K, p.Gp, p.csr_cap, nt);
+    const StreamLayout L(M, p.K, p.Gp, p.csr_cap, nt, p.blk_cap, p.blk_words);
     if (L.total > kMaxSmem) return MQ_ERR_UNSUPPORTED;
     void *kern = M == 1 ? kernel_for<1>(nt) : kernel_for<8>(nt);
     static bool configured[64][2][kTMax + 1] = {};

@@ -403,6 +403,60 @@ mq_status validate_decomp(const mq_decomp *d) {
     return MQ_OK;
 }
 
+bool block_tiles_host(const HostPacked &p, HostBlocks &b) {
+    static const int kPi[8] = {0, 2, 4, 6, 1, 3, 5, 7};
+    b = HostBlocks();
+    const int64_t N = p.N, K = p.K;
+    if (p.nnz == 0 || N % kBlockRows || K % kBlockCols) return false;
+    const int64_t nbr = N / kBlockRows, nbc = K / kBlockCols;
+    std::vector<int32_t> ptr(nbr + 1, 0);
+    std::vector<uint16_t> cols;
+    for (int64_t rb = 0; rb < nbr; ++rb) {
+        const int64_t r0 = rb * kBlockRows;
+        const int64_t len = p.row_ptr[r0 + 1] - p.row_ptr[r0];
+        if (len % kBlockCols) return false;
+        const int64_t nb = len / kBlockCols;
+        for (int64_t r = r0; r < r0 + kBlockRows; ++r) {
+            if (p.row_ptr[r + 1] - p.row_ptr[r] != len) return false;
+            for (int64_t k = 0; k < nb; ++k) {
+                const int64_t e = p.row_ptr[r] + k * kBlockCols;
+                const int64_t c0 = p.col[e];
+                if (c0 % kBlockCols) return false;
+                if (r > r0 && c0 != p.col[p.row_ptr[r0] + k * kBlockCols]) return false;
+                for (int64_t i = 1; i < kBlockCols; ++i)
+                    if (p.col[e + i] != c0 + i) return false;
+            }
+        }
+        for (int64_t k = 0; k < nb; ++k)
+            cols.push_back(static_cast<uint16_t>(p.col[p.row_ptr[r0] + k * kBlockCols] / kBlockCols));
+        ptr[rb + 1] = ptr[rb] + static_cast<int32_t>(nb);
+    }
+    b.nblk = static_cast<int64_t>(cols.size());
+    b.map_words = (nbc + 31) / 32;
+    b.ptr = std::move(ptr);
+    b.col = std::move(cols);
+    b.q.assign(b.nblk * kBlockRows * (kBlockCols / 8), 0);
+    b.map.assign(nbr * b.map_words, 0);
+    for (int64_t rb = 0; rb < nbr; ++rb)
+        for (int64_t k = 0; k < b.ptr[rb + 1] - b.ptr[rb]; ++k) {
+            const int64_t blk = b.ptr[rb] + k, cb = b.col[blk];
+            b.map[rb * b.map_words + cb / 32] |= 1u << (cb % 32);
+            for (int64_t r = 0; r < kBlockRows; ++r) {
+                const int64_t e0 = p.row_ptr[rb * kBlockRows + r] + k * kBlockCols;
+                for (int64_t w = 0; w < kBlockCols / 8; ++w) {
+                    uint32_t word = 0;
+                    for (int j = 0; j < 8; ++j) {
+                        const int64_t e = e0 + 8 * w + kPi[j];
+                        const uint32_t nib = (p.val[e >> 1] >> ((e & 1) * 4)) & 0xF;
+                        word |= ((nib ^ 8u) & 0xF) << (4 * j);  // two's complement -> q_r + 8
+                    }
+                    b.q[(blk * kBlockRows + r) * (kBlockCols / 8) + w] = word;
+                }
+            }
+        }
+    return true;
+}
+
 void pack_host(const mq_decomp &d, HostPacked &p) {
     static const int kPi[8] = {0, 2, 4, 6, 1, 3, 5, 7};
     const int64_t N = d.N, K = d.K, G = K / kGroup;

@@ -45,6 +45,25 @@ struct HostPacked {
     std::vector<uint16_t> rscale;   // [N]
 };
 
+// Block tiles of a residual made of whole 16 x 64 blocks on the block grid
+// (the block allocation): per block-row offsets, column-block indices, and
+// per block 16 rows x 8 words of offset-binary codes q_r + 8 in the base
+// codes' nibble interleave. `map` (device helper, not part of the packed
+// form) has one bit per column-block for every block-row, words of 32.
+struct HostBlocks {
+    int64_t nblk = 0, map_words = 0;
+    std::vector<int32_t> ptr;   // [N/16 + 1]
+    std::vector<uint16_t> col;  // [nblk]
+    std::vector<uint32_t> q;    // [nblk][16][8]
+    std::vector<uint32_t> map;  // [N/16][map_words]
+};
+
+// Builds the tiles when the packed residual is block-structured: N % 16 == 0,
+// K % 64 == 0, and each row of a block-row holds exactly the columns of the
+// same aligned 64-column runs. Returns false (and leaves `b` empty)
+// otherwise, or when there is no residual.
+bool block_tiles_host(const HostPacked &p, HostBlocks &b);
+
 mq_status check_shape(int64_t N, int64_t K, const mq_pack_opts *opts);
 int64_t residual_count(int64_t K, double rho);
 mq_status decompose_host(const float *W, int64_t N, int64_t K, const mq_pack_opts &opts,

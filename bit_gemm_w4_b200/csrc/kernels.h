@@ -45,8 +45,23 @@ struct DeviceWeight {
     const uint16_t *wide_off;  // [ceil(N/128) * S * kWideOffStride]
     const uint16_t *wide_ent;  // [nnz] (+ padding)
     int64_t wide_max;          // longest slice, entries
+    // The residual again as block tiles, when it consists of whole 16 x 64
+    // blocks (block allocation; NULL otherwise): per 16-row block-row the
+    // offsets of its blocks, their column-block indices, 512 bytes of
+    // offset-binary codes q_r + 8 per block (16 rows x 8 words in the base
+    // codes' nibble interleave), and a bitmap of each block-row's column-
+    // blocks (blk_words 32-bit words per block-row).
+    const int32_t *blk_ptr;    // [N/16 + 1]
+    const uint16_t *blk_col;   // [nblk]
+    const uint32_t *blk_q;     // [nblk][16][8]
+    const uint32_t *blk_map;   // [N/16][blk_words]
+    int64_t nblk, blk_words;
     int *err;                 // device error word
 };
+
+// Most blocks over `parts` contiguous runs of 16-row tiles (as for
+// max_span_nnz); 0 when the weight has no block tiles.
+int64_t max_span_blocks(const mq_weight *w, int64_t ntile, int parts);
 
 // Largest residual entry count over the bn-row tiles of a handle (cached per
 // tile height; the decode kernels size their shared-memory CSR slice with it).

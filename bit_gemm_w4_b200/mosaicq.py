@@ -79,6 +79,8 @@ def _load():
         "mq_pack_decomposed": ([ctypes.POINTER(_Decomp), vp, ctypes.POINTER(vp)], st),
         "mq_get_info": ([vp, ctypes.POINTER(_Info)], st),
         "mq_export": ([vp, ctypes.POINTER(_HostPacked)], st),
+        "mq_export_blocks": ([vp, vp, vp, vp, ctypes.POINTER(i64)], st),
+        "mq_block_tiles_host": ([ctypes.POINTER(_Decomp), vp, vp, vp, ctypes.POINTER(i64)], st),
         "mq_device_error": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], st),
         "mq_strerror": ([st], ctypes.c_char_p),
         "mq_last_error": ([], ctypes.c_char_p),
@@ -198,6 +200,37 @@ def selftest_bounded_wait(limit_cycles: int = 1 << 20) -> list:
     return list(out)
 
 
+def _decomp_struct(d: dict, keep: dict) -> "_Decomp":
+    return _Decomp(int(d["N"]), int(d["K"]),
+                   *(_ptr(keep[k]) for k in ("q", "s", "z", "row_ptr", "col", "qr", "sr")))
+
+
+def block_tiles_host(d: dict) -> dict:
+    """The library's host-side block tiles of a decomposition given as arrays
+    (as for Weight.pack_decomposed); MQError with UNSUPPORTED when the
+    residual is not made of whole 16 x 64 blocks."""
+    keep = dict(
+        q=np.ascontiguousarray(d["q"], np.uint8),
+        s=np.ascontiguousarray(np.asarray(d["s"], np.float16).view(np.uint16)),
+        z=np.ascontiguousarray(np.asarray(d["z"], np.float16).view(np.uint16)),
+        row_ptr=np.ascontiguousarray(d["row_ptr"], np.int64),
+        col=np.ascontiguousarray(d["col"], np.int32),
+        qr=np.ascontiguousarray(d["qr"], np.int8),
+        sr=np.ascontiguousarray(np.asarray(d["sr"], np.float16).view(np.uint16)))
+    dc = _decomp_struct(d, keep)
+    n = ctypes.c_int64()
+    _check(_lib.mq_block_tiles_host(ctypes.byref(dc), None, None, None, ctypes.byref(n)),
+           "mq_block_tiles_host")
+    N = int(d["N"])
+    out = dict(blk_ptr=np.zeros(N // 16 + 1, np.int32), blk_col=np.zeros(max(n.value, 1), np.uint16),
+               blk_q=np.zeros((max(n.value, 1), 16, 8), np.uint32))
+    _check(_lib.mq_block_tiles_host(ctypes.byref(dc), _ptr(out["blk_ptr"]), _ptr(out["blk_col"]),
+                                    _ptr(out["blk_q"]), ctypes.byref(n)), "mq_block_tiles_host")
+    out["blk_col"] = out["blk_col"][:n.value]
+    out["blk_q"] = out["blk_q"][:n.value]
+    return out
+
+
 def read_probe(buf_ptr: int, nbytes: int, sink_ptr: int, *, stream=None) -> None:
     """One launch of the library's streaming-read probe (mq_read_probe) over
     nbytes of device memory at buf_ptr; sink_ptr is a 4-byte device word."""
@@ -253,7 +286,7 @@ class Weight:
             col=np.ascontiguousarray(d["col"], np.int32),
             qr=np.ascontiguousarray(d["qr"], np.int8),
             sr=np.ascontiguousarray(np.asarray(d["sr"], np.float16).view(np.uint16)))
-        dc = _Decomp(N, K, *(_ptr(keep[k]) for k in ("q", "s", "z", "row_ptr", "col", "qr", "sr")))
+        dc = _decomp_struct(d, keep)
         h = ctypes.c_void_p()
         _check(_lib.mq_pack_decomposed(ctypes.byref(dc), _stream(stream), ctypes.byref(h)),
                "mq_pack_decomposed")
@@ -338,6 +371,20 @@ class Weight:
         _check(_lib.mq_linear_unfused_noalloc(self._h, X.data_ptr(), X.shape[0], Y.data_ptr(),
                                               _stream(stream)), "mq_linear_unfused_noalloc")
         return Y
+
+    def export_blocks(self) -> dict:
+        """The device copy of the block tiles (blk_ptr, blk_col, blk_q);
+        MQError with UNSUPPORTED when the residual is not block-structured."""
+        n = ctypes.c_int64()
+        _check(_lib.mq_export_blocks(self._h, None, None, None, ctypes.byref(n)), "mq_export_blocks")
+        N = self.info()["N"]
+        out = dict(blk_ptr=np.zeros(N // 16 + 1, np.int32), blk_col=np.zeros(max(n.value, 1), np.uint16),
+                   blk_q=np.zeros((max(n.value, 1), 16, 8), np.uint32))
+        _check(_lib.mq_export_blocks(self._h, _ptr(out["blk_ptr"]), _ptr(out["blk_col"]),
+                                     _ptr(out["blk_q"]), ctypes.byref(n)), "mq_export_blocks")
+        out["blk_col"] = out["blk_col"][:n.value]
+        out["blk_q"] = out["blk_q"][:n.value]
+        return out
 
     def export(self) -> dict:
         info = self.info()

@@ -323,6 +323,32 @@ mq_status mq_get_info(const mq_weight *w, mq_info *out);
  * from mq_get_info). Synchronous: waits for the device. */
 mq_status mq_export(const mq_weight *w, mq_host_packed *out);
 
+/* Block tiles. When a residual consists of whole 16-row x 64-column blocks
+ * on the block grid (the block allocation of "Methodology" 2., Block-Wise
+ * Residual Allocation: mq_pack with residual_blocks = 1, or such a
+ * decomposition given to mq_pack_decomposed), the library also holds it as
+ * block tiles, which the decode kernels run as extra tensor-core passes:
+ *   blk_ptr i32 [N/16 + 1]: offsets of each 16-row block-row's blocks;
+ *   blk_col u16 [nblk]: the column-block index cb of each block (columns
+ *     64*cb .. 64*cb + 63), ascending within a block-row;
+ *   blk_q u32 [nblk][16][8]: word w of row r holds, in bits [4j, 4j+4),
+ *     u = q_r + 8 (offset binary 0..15) of column 64*cb + 8w + pi(j),
+ *     pi = (0,2,4,6,1,3,5,7) as for qweight.
+ * The CSR (mq_export) holds the same codes.
+ *
+ * mq_block_tiles_host computes the tiles of a decomposition on the host (no
+ * CUDA call); mq_export_blocks copies a packed weight's tiles to the host
+ * (synchronizing its device). Both write *nblk; with blk_ptr = NULL they
+ * stop there (a size query), else the three caller-owned buffers must hold
+ * N/16 + 1, nblk and nblk * 128 elements.
+ * Errors: INVALID_ARG for a NULL d/w or nblk, a NULL buffer when blk_ptr is
+ * given, or an invalid decomposition; UNSUPPORTED when the residual is not
+ * made of whole blocks (or is empty); CUDA for a failed copy. */
+mq_status mq_block_tiles_host(const mq_decomp *d, int32_t *blk_ptr, uint16_t *blk_col,
+                              uint32_t *blk_q, int64_t *nblk);
+mq_status mq_export_blocks(const mq_weight *w, int32_t *blk_ptr, uint16_t *blk_col,
+                           uint32_t *blk_q, int64_t *nblk);
+
 /* Read and clear the handle's device error word: 0 when every kernel since
  * the last read finished its waits, else the code of the wait that gave up.
  * Synchronizes `stream`. Returns MQ_ERR_DEVICE_TIMEOUT when non-zero. */

@@ -263,6 +263,33 @@ def test_block_mode_parity(mq, cuda, M):
     assert r["ok"], r
 
 
+@pytest.mark.parametrize("N,K,M", [(4096, 4096, 1), (4096, 4096, 8), (2048, 11008, 3)])
+def test_block_tiles_decode(mq, cuda, N, K, M):
+    # a block-allocated residual held as block tiles (byte-exact with the
+    # oracle's layout) and run as tensor-core passes by the streaming decode
+    # kernel, several tiles per CTA
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=N + M)
+    w = mq.Weight.pack(W, block_fraction=0.1)
+    d = oracle.decompose_blocks(W, 0.1)
+    want = oracle.pack_blocks(d)
+    got = w.export_blocks()
+    for k in ("blk_ptr", "blk_col", "blk_q"):
+        assert np.array_equal(np.asarray(got[k]).view(np.uint8), np.asarray(want[k]).view(np.uint8)), k
+    X = synth.activations(M, K, seed=50 + M, channels=4, mult=20.0)
+    Y = w.linear(X.cuda())
+    torch.cuda.synchronize()
+    assert w.device_error() == 0
+    r = oracle_check(Y, X, d)
+    assert r["ok"], r
+
+
+def test_block_tiles_absent_for_row_residuals(mq, cuda):
+    w = mq.Weight.pack(synth.weight(64, 256, std=0.02, outlier_frac=0.005, seed=1), 0.05)
+    with pytest.raises(mq.MQError) as e:
+        w.export_blocks()
+    assert e.value.status == mq.UNSUPPORTED
+
+
 def test_block_mode_long_rows(mq, cuda):
     # 10 % of the 16 x 64 blocks of a 1024 x 11008 projection carry a residual
     N, K = 1024, 11008

@@ -106,3 +106,26 @@ def test_block_mode_counts_and_errors(mq):
     with pytest.raises(mq.MQError) as e:
         mq.pack_host(W, 0.0, block_fraction=2.0)
     assert e.value.status == 1
+
+
+def _arrays(d):
+    return dict(N=d.N, K=d.K, q=d.q, s=d.s, z=d.z, row_ptr=d.row_ptr, col=d.col, qr=d.qr, sr=d.sr)
+
+
+@pytest.mark.parametrize("N,K,frac", [(32, 256, 0.1), (64, 512, 0.03), (48, 1024, 0.5), (16, 128, 1.0)])
+def test_block_tiles_equal_oracle(mq, N, K, frac):
+    # the library's block tiles of a block-allocated residual, byte for byte
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=N + K)
+    d = oracle.decompose_blocks(W, frac)
+    got = mq.block_tiles_host(_arrays(d))
+    want = oracle.pack_blocks(d)
+    for k in ("blk_ptr", "blk_col", "blk_q"):
+        a, b = np.asarray(got[k]), np.asarray(want[k])
+        assert a.shape == b.shape and np.array_equal(a.view(np.uint8), b.view(np.uint8)), k
+
+
+def test_block_tiles_refuse_a_row_residual(mq):
+    d = oracle.decompose(synth.weight(32, 256, std=0.02, outlier_frac=0.005, seed=2), 0.05)
+    with pytest.raises(mq.MQError) as e:
+        mq.block_tiles_host(_arrays(d))
+    assert e.value.status == mq.UNSUPPORTED
