@@ -65,12 +65,12 @@ def alg_bytes(M: int, N: int, K: int, nnz: int) -> int:
             + 2 * M * K + 2 * M * N)
 
 
-# DRAM bytes (read + write) of one decode launch, 4096 x 4096, M = 1, density
-# 0.5 %, from one ncu capture of the current decode kernel (the summary under
-# profiles/ gives the command). The bench's other shapes are scaled by their
-# packed size N*K, which the traffic follows (no re-reads). Set to None when
-# the decode kernel changes until it is captured again.
-DECODE_TRAFFIC_4096 = None
+# DRAM bytes (read + write) of one launch of the streaming decode kernel per
+# 7B shape (M = 1, density 0.5 %), each from one ncu capture of that shape
+# (profiles/decode_stream_kernel_7b_m1.txt gives the commands). Set to None
+# when the kernel changes until it is captured again.
+DECODE_TRAFFIC = {(4096, 4096): 9.223168e6, (11008, 4096): 24.663808e6,
+                  (4096, 11008): 24.668928e6}
 
 
 def alg_flops(M: int, N: int, K: int, nnz: int) -> int:
@@ -545,11 +545,11 @@ def run_ours(args):
                    "parallelism": f"replicas x{dist_ctx.world}", "timing": "CUDA graph replay"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
-                     "traffic": (None if DECODE_TRAFFIC_4096 is None else
-                                 round(sum(DECODE_TRAFFIC_4096 * N * K / 4096 ** 2
+                     "traffic": (None if DECODE_TRAFFIC is None else
+                                 round(sum(DECODE_TRAFFIC[(N, K)]
                                            for N, K in ds.shapes))),
-                     "traffic_note": "DRAM bytes per step (3 launches): one ncu capture of the "
-                                     "4096x4096 launch scaled by N*K",
+                     "traffic_note": "DRAM bytes per step (3 launches): the sum of one ncu "
+                                     "capture of each shape's launch",
                      "peak_source": pk_src,
                      "spec_gbs": SPEC_HBM_GBS,
                      "frac_of_spec": round(achieved / SPEC_HBM_GBS, 4),
@@ -557,7 +557,7 @@ def run_ours(args):
                      "frac_of_read_ceiling": round(achieved / read_ceiling, 4),
                      "read_ceiling_note": "mq_read_probe over the step's three per-launch byte "
                                           "counts, rotated and replayed like the step",
-                     "kernel": "decode_kernel (the step's three launches)",
+                     "kernel": "decode_stream_kernel (the step's three launches)",
                      "per_shape_us": {f"{N}x{K}": round(t * 1e3, 3)
                                       for (N, K), t in zip(ds.shapes, per_shape)},
                      "per_shape_frac": {f"{N}x{K}": round(b / (t * 1e-3) / 1e9 / pk["hbm_gbs"], 4)
@@ -659,6 +659,7 @@ PROFILE_CASES = {
     # name: (N, K, M, rho, path)
     "decode-4096x4096-m1": (4096, 4096, 1, 0.005, "auto"),
     "decode-11008x4096-m1": (11008, 4096, 1, 0.005, "auto"),
+    "decode-4096x11008-m1": (4096, 11008, 1, 0.005, "auto"),
     "decode-28672x8192-m16": (28672, 8192, 16, 0.01, "auto"),
     "prefill-14336x4096-m256": (14336, 4096, 256, 0.005, "prefill"),
     "prefill-14336x4096-m2048": (14336, 4096, 2048, 0.005, "prefill"),
