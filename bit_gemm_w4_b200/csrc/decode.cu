@@ -461,7 +461,10 @@ mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaS
         const mq_status st = launch_decode_wide(w, X, M, Y, stream, partial, pf);
         if (st != MQ_ERR_UNSUPPORTED) return st;
     }
-    if (M <= 8) {
+    {
+        // the streaming kernel, when X (and a CTA's residual share) fits its
+        // shared memory: up to 16 tokens (9-16 only on layers the wide kernel
+        // above did not take)
         const mq_status st = launch_decode_stream(w, X, M, Y, stream, partial, pf);
         if (st != MQ_ERR_UNSUPPORTED) return st;
     }

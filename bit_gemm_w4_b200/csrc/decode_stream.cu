@@ -62,14 +62,16 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTMax = 8;     // most tiles per CTA (one accumulator set each)
-constexpr int kMaxSmem = 200 * 1024;
+constexpr int kMaxSmem = 227 * 1024;
 constexpr int kCsrBudget = 24 * 1024;    // shared memory for a CTA's CSR slice
 constexpr int kBlockBudget = 48 * 1024;  // shared memory for a CTA's block tiles
 
 // Groups of prefetch ahead for NT tiles per CTA: eight to ten items per
-// thread (64-80 KB per CTA in flight), or one group for NT > 5.
-__host__ __device__ constexpr int groups_ahead(int nt) {
-    return nt >= 6 ? 1 : nt >= 4 ? 2 : nt == 3 ? 3 : nt == 2 ? 4 : 8;
+// thread (64-80 KB per CTA in flight), or one group for NT > 5; half as many
+// at 16 tokens, where X takes most of the shared memory.
+__host__ __device__ constexpr int groups_ahead(int nt, bool wide_x = false) {
+    return wide_x ? (nt >= 3 ? 1 : nt == 2 ? 2 : 4)
+                  : (nt >= 6 ? 1 : nt >= 4 ? 2 : nt == 3 ? 3 : nt == 2 ? 4 : 8);
 }
 
 struct StreamParams {
@@ -107,8 +109,8 @@ struct StreamLayout {
     int ring, x, xrs, szs, red, res, rsf, rp, col, val, bq, bmap, bpre, total;
     __host__ __device__ StreamLayout(int M, int K, int Gp, int csr_cap, int nt, int blk_cap = 0,
                                      int blk_words = 0) {
-        ring = 0;                                              // [D * NT][2][kThreads][16 B]
-        x = ring + groups_ahead(nt) * nt * 2 * kThreads * 16;  // [M][xrs]
+        ring = 0;                                                       // [D * NT][2][kThreads][16 B]
+        x = ring + groups_ahead(nt, M > 8) * nt * 2 * kThreads * 16;   // [M][xrs]
         xrs = K * 2 + 16;
         szs = x + (M * xrs + 15) / 16 * 16;                    // [NT * 16][sz_stride] words
         red = szs + nt * 16 * sz_stride(Gp) * 4;               // [NT][warp][M][16] fp32
@@ -160,9 +162,10 @@ __device__ __forceinline__ void mma_pure(float (&d)[4], const uint32_t (&a)[4], 
 }
 
 
-template <int MX, int NT>
+template <int MX, int NT, bool BLK>
 __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid_constant__ StreamParams p) {
-    constexpr int D = groups_ahead(NT);
+    constexpr int NTOK = MX > 8 ? 2 : 1;  // 8-token MMA column tiles
+    constexpr int D = groups_ahead(NT, MX > 8);
     constexpr int R = D * NT;  // ring slots (items) per thread
     extern __shared__ __align__(16) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,7 +179,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
     const bool full = nt == NT;  // only tile NT - 1 can be missing
     const int gpw = warp < G ? (G - warp + kWarps - 1) / kWarps : 0;  // groups of this warp
     const bool resid = p.csr_cap > 0;
-    const bool blocks = p.blk_cap > 0;
+    // the block-tile residual path exists only in its own instantiations, so
+    // that the row-residual kernels carry none of its code
+    constexpr bool blocks = BLK;
 
     // ------------------------------------------------ the weight stream
     // Row offsets (words) of this thread's rows g and g+8 in each tile, and
@@ -287,15 +292,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
     float *res = reinterpret_cast<float *>(smem + L.res);
 
     // ------------------------------------------------ dense pass
-    float acc[NT][4];
+    float acc[NT][NTOK][4];
 #pragma unroll
     for (int k = 0; k < NT; ++k)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[k][i] = 0.f;
-    uint32_t xb[16];
+        for (int n8 = 0; n8 < NTOK; ++n8)
 #pragma unroll
-    for (int i = 0; i < 16; ++i) xb[i] = 0u;
-    const bool xlane = MX == 1 ? g == 0 : g < M;  // lanes whose token column is live
+            for (int i = 0; i < 4; ++i) acc[k][n8][i] = 0.f;
+    uint32_t xb[NTOK][16];
+#pragma unroll
+    for (int n8 = 0; n8 < NTOK; ++n8)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xb[n8][i] = 0u;
 #pragma unroll 1
     for (int j0 = 0; j0 < gpw; j0 += D) {
 #pragma unroll
@@ -303,17 +311,47 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
             const int j = j0 + d;
             if (j < gpw) {
                 const int gi = warp + kWarps * j;
-                if (xlane) {
-                    const uint8_t *xp = xs + g * L.xrs + gi * 256;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(xp + xchunk(4 * t + i) * 16);
-                        xb[4 * i + 0] = v.x;
-                        xb[4 * i + 1] = v.y;
-                        xb[4 * i + 2] = v.z;
-                        xb[4 * i + 3] = v.w;
+                for (int n8 = 0; n8 < NTOK; ++n8) {
+                    const int tok = g + 8 * n8;
+                    // lanes whose token column is live
+                    if (MX == 1 ? g == 0 : tok < M) {
+                        const uint8_t *xp = xs + tok * L.xrs + gi * 256;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(xp + xchunk(4 * t + i) * 16);
+                            xb[n8][4 * i + 0] = v.x;
+                            xb[n8][4 * i + 1] = v.y;
+                            xb[n8][4 * i + 2] = v.z;
+                            xb[n8][4 * i + 3] = v.w;
+                        }
                     }
                 }
+                // k-step ks of the group for every 8-token tile: even steps into
+                // ca, odd ones into cb (two independent accumulator chains)
+                auto mma_acc = [&](float (&ca)[NTOK][4], float (&cb)[NTOK][4], const uint32_t (&a)[4],
+                                   int ks) {
+#pragma unroll
+                    for (int n8 = 0; n8 < NTOK; ++n8) {
+                        if (ks & 1)
+                            mma_pure(cb[n8], a, xb[n8][2 * ks], xb[n8][2 * ks + 1]);
+                        else
+                            mma_pure(ca[n8], a, xb[n8][2 * ks], xb[n8][2 * ks + 1]);
+                    }
+                };
+                // acc[k] += scale * partial, rows g (scale s0) and g + 8 (s1)
+                auto scale_add = [&](int k, const float (&ca)[NTOK][4], const float (&cb)[NTOK][4],
+                                     float s0, float s1) {
+#pragma unroll
+                    for (int n8 = 0; n8 < NTOK; ++n8) {
+                        acc[k][n8][0] = fmaf(s0, ca[n8][0] + cb[n8][0], acc[k][n8][0]);
+                        acc[k][n8][2] = fmaf(s1, ca[n8][2] + cb[n8][2], acc[k][n8][2]);
+                        if (MX > 1) {  // token columns 2t + 1 (none live at one token)
+                            acc[k][n8][1] = fmaf(s0, ca[n8][1] + cb[n8][1], acc[k][n8][1]);
+                            acc[k][n8][3] = fmaf(s1, ca[n8][3] + cb[n8][3], acc[k][n8][3]);
+                        }
+                    }
+                };
                 // the residual blocks of tile k in group gi (column-blocks 2gi and
                 // 2gi + 1; lanes t = 0, 1 hold the first, t = 2, 3 the second):
                 // one more pass over the group's X fragment with offset-binary
@@ -336,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
                     }
                     const uint32_t bias = p.bias;
                     const uint32_t zz = 0x43084308u;  // bf16x2 (136, 136): u - 8 = q_r exactly
-                    float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+                    float ca[NTOK][4] = {}, cb[NTOK][4] = {};
                     const uint32_t wr0[4] = {ba.x, ba.y, ba.z, ba.w};
                     const uint32_t wr1[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
@@ -348,18 +386,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
                         a[1] = bf16x2_sub(nib_pair(b_lo, bias), zz);
                         a[2] = bf16x2_sub(nib_pair(a_lo >> 4, bias), zz);
                         a[3] = bf16x2_sub(nib_pair(b_lo >> 4, bias), zz);
-                        if (ks & 1)
-                            mma_pure(cb, a, xb[2 * ks], xb[2 * ks + 1]);
-                        else
-                            mma_pure(ca, a, xb[2 * ks], xb[2 * ks + 1]);
+                        mma_acc(ca, cb, a, ks);
                     }
-                    const float r0s = rsfs[k * 16 + g], r1s = rsfs[k * 16 + g + 8];
-                    acc[k][0] = fmaf(r0s, ca[0] + cb[0], acc[k][0]);
-                    acc[k][2] = fmaf(r1s, ca[2] + cb[2], acc[k][2]);
-                    if (MX > 1) {
-                        acc[k][1] = fmaf(r0s, ca[1] + cb[1], acc[k][1]);
-                        acc[k][3] = fmaf(r1s, ca[3] + cb[3], acc[k][3]);
-                    }
+                    scale_add(k, ca, cb, rsfs[k * 16 + g], rsfs[k * 16 + g + 8]);
                 };
                 // one item: tile k of group gi, from ring slot d * NT + k
                 auto item = [&](int k) {
@@ -370,8 +399,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
                     const uint32_t sz1 = szs[(k * 16 + g + 8) * SZS + gi];
                     const uint32_t zz0 = zero_pair(sz0), zz1 = zero_pair(sz1);
                     const uint32_t bias = p.bias;
-                    // two accumulator chains (even and odd k-steps)
-                    float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+                    // two accumulator chains (even and odd k-steps) per token tile
+                    float ca[NTOK][4] = {}, cb[NTOK][4] = {};
                     const uint32_t wr0[4] = {wa.x, wa.y, wa.z, wa.w};
                     const uint32_t wr1[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
@@ -383,19 +412,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
                         a[1] = bf16x2_sub(nib_pair(b_lo, bias), zz1);
                         a[2] = bf16x2_sub(nib_pair(a_lo >> 4, bias), zz0);
                         a[3] = bf16x2_sub(nib_pair(b_lo >> 4, bias), zz1);
-                        if (ks & 1)
-                            mma_pure(cb, a, xb[2 * ks], xb[2 * ks + 1]);
-                        else
-                            mma_pure(ca, a, xb[2 * ks], xb[2 * ks + 1]);
+                        mma_acc(ca, cb, a, ks);
                     }
-                    const float s0 = half_bits_to_f32(sz0), s1 = half_bits_to_f32(sz1);
-                    acc[k][0] = fmaf(s0, ca[0] + cb[0], acc[k][0]);
-                    acc[k][2] = fmaf(s1, ca[2] + cb[2], acc[k][2]);
-                    if (MX > 1) {  // token columns 2t + 1 (none live at one token)
-                        acc[k][1] = fmaf(s0, ca[1] + cb[1], acc[k][1]);
-                        acc[k][3] = fmaf(s1, ca[3] + cb[3], acc[k][3]);
-                    }
-                    if (blocks) block_pass(k, gi);
+                    scale_add(k, ca, cb, half_bits_to_f32(sz0), half_bits_to_f32(sz1));
+                    if constexpr (BLK) block_pass(k, gi);
                 };
                 // items in pairs after one wait, so that the two interleave;
                 // each slot is refilled D groups ahead once its values are used
@@ -421,13 +441,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
     for (int k = 0; k < NT; ++k) {
         if (k < nt) {
             float *rw = red + ((k * kWarps + warp) * M) * 16;
-            if (2 * t < M) {
-                rw[(2 * t) * 16 + g] = acc[k][0];
-                rw[(2 * t) * 16 + g + 8] = acc[k][2];
-            }
-            if (MX > 1 && 2 * t + 1 < M) {
-                rw[(2 * t + 1) * 16 + g] = acc[k][1];
-                rw[(2 * t + 1) * 16 + g + 8] = acc[k][3];
+#pragma unroll
+            for (int n8 = 0; n8 < NTOK; ++n8) {
+                const int m0 = 8 * n8 + 2 * t;
+                if (m0 < M) {
+                    rw[m0 * 16 + g] = acc[k][n8][0];
+                    rw[m0 * 16 + g + 8] = acc[k][n8][2];
+                }
+                if (MX > 1 && m0 + 1 < M) {
+                    rw[(m0 + 1) * 16 + g] = acc[k][n8][1];
+                    rw[(m0 + 1) * 16 + g + 8] = acc[k][n8][3];
+                }
             }
         }
     }
@@ -528,17 +552,27 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
     cp_async_wait_all();
 }
 
-template <int MX>
+template <int MX, bool BLK>
 void *kernel_for(int nt) {
-    switch (nt) {
-        case 1: return reinterpret_cast<void *>(decode_stream_kernel<MX, 1>);
-        case 2: return reinterpret_cast<void *>(decode_stream_kernel<MX, 2>);
-        case 3: return reinterpret_cast<void *>(decode_stream_kernel<MX, 3>);
-        case 4: return reinterpret_cast<void *>(decode_stream_kernel<MX, 4>);
-        case 5: return reinterpret_cast<void *>(decode_stream_kernel<MX, 5>);
-        case 6: return reinterpret_cast<void *>(decode_stream_kernel<MX, 6>);
-        case 7: return reinterpret_cast<void *>(decode_stream_kernel<MX, 7>);
-        default: return reinterpret_cast<void *>(decode_stream_kernel<MX, 8>);
+    if constexpr (MX > 8) {  // 16 tokens: X takes the shared memory of more tiles
+        switch (nt) {
+            case 1: return reinterpret_cast<void *>(decode_stream_kernel<MX, 1, BLK>);
+            case 2: return reinterpret_cast<void *>(decode_stream_kernel<MX, 2, BLK>);
+            case 3: return reinterpret_cast<void *>(decode_stream_kernel<MX, 3, BLK>);
+            case 4: return reinterpret_cast<void *>(decode_stream_kernel<MX, 4, BLK>);
+            default: return nullptr;
+        }
+    } else {
+        switch (nt) {
+            case 1: return reinterpret_cast<void *>(decode_stream_kernel<MX, 1, BLK>);
+            case 2: return reinterpret_cast<void *>(decode_stream_kernel<MX, 2, BLK>);
+            case 3: return reinterpret_cast<void *>(decode_stream_kernel<MX, 3, BLK>);
+            case 4: return reinterpret_cast<void *>(decode_stream_kernel<MX, 4, BLK>);
+            case 5: return reinterpret_cast<void *>(decode_stream_kernel<MX, 5, BLK>);
+            case 6: return reinterpret_cast<void *>(decode_stream_kernel<MX, 6, BLK>);
+            case 7: return reinterpret_cast<void *>(decode_stream_kernel<MX, 7, BLK>);
+            default: return reinterpret_cast<void *>(decode_stream_kernel<MX, 8, BLK>);
+        }
     }
 }
 
@@ -547,7 +581,7 @@ void *kernel_for(int nt) {
 mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y,
                                cudaStream_t stream, float *partial, const L2Prefetch &pf) {
     const DeviceWeight &d = weight_device(w);
-    if (M < 1 || M > 8) return MQ_ERR_UNSUPPORTED;
+    if (M < 1 || M > 16) return MQ_ERR_UNSUPPORTED;
     const int64_t ntile = (d.N + 15) / 16;
     // one CTA per SM with NT = ceil(tiles / SMs) tiles each, or more CTAs of
     // kTMax tiles for layers taller than kTMax tiles per SM
@@ -589,11 +623,16 @@ mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y
     p.pf = pf;
     const StreamLayout L(M, p.K, p.Gp, p.csr_cap, nt, p.blk_cap, p.blk_words);
     if (L.total > kMaxSmem) return MQ_ERR_UNSUPPORTED;
-    void *kern = M == 1 ? kernel_for<1>(nt) : kernel_for<8>(nt);
-    static bool configured[64][2][kTMax + 1] = {};
+    const int mx = M == 1 ? 0 : M <= 8 ? 1 : 2;
+    void *kern = use_blocks ? (mx == 0 ? kernel_for<1, true>(nt) : mx == 1 ? kernel_for<8, true>(nt)
+                                                                         : kernel_for<16, true>(nt))
+                            : (mx == 0 ? kernel_for<1, false>(nt) : mx == 1 ? kernel_for<8, false>(nt)
+                                                                           : kernel_for<16, false>(nt));
+    if (!kern) return MQ_ERR_UNSUPPORTED;
+    static bool configured[64][2][3][kTMax + 1] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(MQ_ERR_CUDA, "cudaGetDevice failed");
-    if (dev >= 0 && dev < 64 && !configured[dev][M > 1][nt]) {
+    if (dev >= 0 && dev < 64 && !configured[dev][use_blocks][mx][nt]) {
         // the largest shared-memory carveout for every decode kernel, so that
         // consecutive launches of different layers can share an SM without
         // waiting for it to drain and be reconfigured
@@ -602,7 +641,7 @@ mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y
             cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return fail(MQ_ERR_CUDA, "cudaFuncSetAttribute failed for the streaming decode kernel");
-        configured[dev][M > 1][nt] = true;
+        configured[dev][use_blocks][mx][nt] = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
