@@ -160,6 +160,34 @@ void build_wide_lists(const HostPacked &hp, std::vector<int32_t> &ptr, std::vect
         }
 }
 
+// The residual grouped per (16-row tile, 128-column group, half-group) for
+// the tall-layer decode kernel (layout in kernels.h, DeviceWeight::tl_ptr).
+// The half-group of column c is (c % 32) / 16: under the nibble interleave,
+// MMA k-step (c % 32) / 4 covers c, so each half holds four of the group's
+// eight k-steps. An entry is stored as the byte where its code goes in the
+// half's four m16n8k16 A-fragment tiles (512 bytes each; inside one, thread
+// (g = r % 8, t = c / 32) holds it in register (r / 8) + 2 * ((c % 4) / 2),
+// half c % 2), with the stored nibble above it.
+void build_tile_lists(const HostPacked &hp, std::vector<int32_t> &ptr, std::vector<uint16_t> &ent) {
+    const int64_t tiles = (hp.N + 15) / 16, G = hp.K / 128, keys = tiles * G * 2;
+    auto key = [&](int64_t n, int64_t c) { return ((n / 16) * G + c / 128) * 2 + (c % 32) / 16; };
+    ptr.assign(static_cast<size_t>(keys + 1), 0);
+    for (int64_t n = 0; n < hp.N; ++n)
+        for (int64_t e = hp.row_ptr[n]; e < hp.row_ptr[n + 1]; ++e) ++ptr[key(n, hp.col[e]) + 1];
+    for (int64_t k = 0; k < keys; ++k) ptr[k + 1] += ptr[k];
+    ent.assign(static_cast<size_t>(hp.nnz), 0);
+    std::vector<int32_t> fill(ptr.begin(), ptr.end() - 1);
+    for (int64_t n = 0; n < hp.N; ++n)
+        for (int64_t e = hp.row_ptr[n]; e < hp.row_ptr[n + 1]; ++e) {
+            const int64_t c = hp.col[e];
+            const uint32_t nib = (hp.val[e >> 1] >> ((e & 1) * 4)) & 0xF;
+            const int64_t r = n % 16, cg = c % 128;
+            const int64_t pos = ((cg % 32) / 4 % 4) * 512 +
+                                (((r % 8) * 4 + cg / 32) * 4 + r / 8 + 2 * ((cg % 4) / 2)) * 4 + (cg % 2) * 2;
+            ent[fill[key(n, c)]++] = static_cast<uint16_t>(pos | (nib << 11));
+        }
+}
+
 mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **out) {
     *out = nullptr;
     // Failure injection for tests: MQ_FAULT_ALLOC=1 makes the first device
@@ -211,6 +239,15 @@ mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **o
         if (!st) st = upload(w, &woff, hwoff.data(), hwoff.size(), 0, stream);
         if (!st) st = upload(w, &went, hwent.data(), hwent.size(), 64, stream);
     }
+    int32_t *tptr = nullptr;
+    uint16_t *tent = nullptr;
+    if (!st && hp.nnz > 0) {
+        std::vector<int32_t> htptr;
+        std::vector<uint16_t> htent;
+        build_tile_lists(hp, htptr, htent);
+        st = upload(w, &tptr, htptr.data(), htptr.size(), 0, stream);
+        if (!st) st = upload(w, &tent, htent.data(), htent.size(), 64, stream);
+    }
     int32_t *bptr = nullptr;
     uint16_t *bcol = nullptr;
     uint32_t *bq = nullptr, *bmap = nullptr;
@@ -242,6 +279,8 @@ mq_status upload_packed(const HostPacked &hp, cudaStream_t stream, mq_weight **o
     d.wide_off = woff;
     d.wide_ent = went;
     d.wide_max = wide_max;
+    d.tl_ptr = tptr;
+    d.tl_ent = tent;
     d.blk_ptr = bptr;
     d.blk_col = bcol;
     d.blk_q = bq;
@@ -446,6 +485,32 @@ mq_status mq_prefill_lists_host(int64_t N, int64_t K, const int32_t *row_ptr, co
     build_stage_lists(hp, hptr, hent);
     std::memcpy(ptr, hptr.data(), hptr.size() * 4);
     if (nnz) std::memcpy(ent, hent.data(), hent.size() * 4);
+    return MQ_OK;
+}
+
+mq_status mq_tile_lists_host(int64_t N, int64_t K, const int32_t *row_ptr, const uint16_t *col,
+                             const uint8_t *val, int32_t *ptr, uint16_t *ent) {
+    if (N <= 0 || K <= 0 || K % 128) return fail(MQ_ERR_INVALID_ARG, "N, K: positive, K a multiple of 128");
+    if (!row_ptr || !ptr) return fail(MQ_ERR_INVALID_ARG, "a buffer is NULL");
+    const int64_t nnz = row_ptr[N];
+    if (row_ptr[0] != 0 || nnz < 0) return fail(MQ_ERR_INVALID_ARG, "row_ptr must start at 0");
+    for (int64_t n = 0; n < N; ++n)
+        if (row_ptr[n + 1] < row_ptr[n]) return fail(MQ_ERR_INVALID_ARG, "row_ptr must not decrease");
+    if (nnz > 0 && (!col || !val || !ent)) return fail(MQ_ERR_INVALID_ARG, "col, val or ent is NULL");
+    for (int64_t e = 0; e < nnz; ++e)
+        if (col[e] >= K) return fail(MQ_ERR_INVALID_ARG, "a column is not below K");
+    HostPacked hp;
+    hp.N = N;
+    hp.K = K;
+    hp.nnz = nnz;
+    hp.row_ptr.assign(row_ptr, row_ptr + N + 1);
+    hp.col.assign(col, col + nnz);
+    hp.val.assign(val, val + (nnz + 1) / 2);
+    std::vector<int32_t> hptr;
+    std::vector<uint16_t> hent;
+    build_tile_lists(hp, hptr, hent);
+    std::memcpy(ptr, hptr.data(), hptr.size() * 4);
+    if (nnz) std::memcpy(ent, hent.data(), hent.size() * 2);
     return MQ_OK;
 }
 

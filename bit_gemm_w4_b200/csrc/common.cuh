@@ -342,4 +342,55 @@ __device__ __forceinline__ uint4 lds128(const void *p) {
     return v;
 }
 
+// ---- shared by the streaming decode kernels
+
+// bf16x2 (128 + q_lo, 128 + q_hi) for the nibbles at bits [0,4) and [16,20)
+// of w, with the bias word in a register: one LOP3.
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, uint32_t bias) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(0x000F000F), "r"(bias));
+    return d;
+}
+
+// bf16x2 (128 + z, 128 + z) from a scale/zero word (fp16 s low, fp16 z high,
+// z an integer 0..15): adding 1024 in fp16 puts z in the low mantissa bits.
+__device__ __forceinline__ uint32_t zero_pair(uint32_t szw) {
+    uint32_t h;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(h) : "r"(szw), "r"(0x64006400u));
+    return (__byte_perm(h, 0, 0x3232) & 0x000F000Fu) | 0x43004300u;
+}
+
+// cp.async of 16 bytes, or of none (zero fill) when `live` is false.
+__device__ __forceinline__ void cp_async16_if(void *dst, const void *src, bool live) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(live ? 16 : 0)
+                 : "memory");
+}
+
+// D += A * B, m16n8k16 bf16 -> fp32, as a pure function of its operands (not
+// volatile), so that the compiler may interleave independent items.
+__device__ __forceinline__ void mma_pure(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// scale/zero row stride in shared memory (words): Gp, or Gp + 4, whichever
+// is an odd multiple of four
+__host__ __device__ inline int sz_stride(int Gp) { return ((Gp >> 2) & 1) ? Gp : Gp + 4; }
+
+// 16-byte chunk c of a 128-column group of X sits at xchunk(c) in shared
+// memory, so that a warp's fragment loads touch distinct banks.
+__device__ __forceinline__ int xchunk(int c) { return c ^ (((c >> 3) & 1) << 1); }
+
+// Byte offset in a fragment tile of the code at row r (0..15), column c of a
+// 128-column group: thread (g = r % 8, t = c / 32) holds it in register
+// (r / 8) + 2 * ((c % 4) / 2), half c % 2 (the m16n8k16 A layout under the
+// packed codes' k order, where k-step (c % 32) / 4 covers column c).
+__device__ __forceinline__ int tile_pos(int r, int c) {
+    return (((r & 7) * 4 + (c >> 5)) * 4 + (r >> 3) + 2 * ((c & 3) >> 1)) * 4 + (c & 1) * 2;
+}
+
 }  // namespace mq

@@ -457,15 +457,19 @@ mq_status run_cs(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t
 
 mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t stream,
                         float *partial, const L2Prefetch &pf) {
-    if (M > 8) {
-        const mq_status st = launch_decode_wide(w, X, M, Y, stream, partial, pf);
-        if (st != MQ_ERR_UNSUPPORTED) return st;
-    }
     {
         // the streaming kernel, when X (and a CTA's residual share) fits its
-        // shared memory: up to 16 tokens (9-16 only on layers the wide kernel
-        // above did not take)
+        // shared memory without leaving a second wave of CTAs
         const mq_status st = launch_decode_stream(w, X, M, Y, stream, partial, pf);
+        if (st != MQ_ERR_UNSUPPORTED) return st;
+    }
+    if (M > 1) {
+        // tall layers whose X does not fit: X from L2
+        const mq_status st = launch_decode_tall(w, X, M, Y, stream, partial, pf);
+        if (st != MQ_ERR_UNSUPPORTED) return st;
+    }
+    if (M > 8) {
+        const mq_status st = launch_decode_wide(w, X, M, Y, stream, partial, pf);
         if (st != MQ_ERR_UNSUPPORTED) return st;
     }
     if (M == 1) {

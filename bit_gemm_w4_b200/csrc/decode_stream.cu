@@ -63,6 +63,7 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTMax = 8;     // most tiles per CTA (one accumulator set each)
 constexpr int kMaxSmem = 227 * 1024;
+constexpr int kTwoPerSm = 113 * 1024;  // shared memory of each of two CTAs per SM
 constexpr int kCsrBudget = 24 * 1024;    // shared memory for a CTA's CSR slice
 constexpr int kBlockBudget = 48 * 1024;  // shared memory for a CTA's block tiles
 
@@ -100,9 +101,6 @@ struct StreamParams {
     L2Prefetch pf;  // another weight, brought into L2 meanwhile
 };
 
-// scale/zero row stride in shared memory (words): Gp, or Gp + 4, whichever
-// is an odd multiple of four
-__host__ __device__ inline int sz_stride(int Gp) { return ((Gp >> 2) & 1) ? Gp : Gp + 4; }
 
 // Shared-memory layout (bytes), identical on host and device.
 struct StreamLayout {
@@ -126,40 +124,6 @@ struct StreamLayout {
     }
 };
 
-// bf16x2 (128 + q_lo, 128 + q_hi) for the nibbles at bits [0,4) and [16,20)
-// of w, with the bias word in a register: one LOP3.
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w, uint32_t bias) {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(0x000F000F), "r"(bias));
-    return d;
-}
-
-// bf16x2 (128 + z, 128 + z) from a scale/zero word (fp16 s low, fp16 z high,
-// z an integer 0..15): adding 1024 in fp16 puts z in the low mantissa bits.
-__device__ __forceinline__ uint32_t zero_pair(uint32_t szw) {
-    uint32_t h;
-    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(h) : "r"(szw), "r"(0x64006400u));
-    return (__byte_perm(h, 0, 0x3232) & 0x000F000Fu) | 0x43004300u;
-}
-
-// cp.async of 16 bytes, or of none (zero fill) when `live` is false.
-__device__ __forceinline__ void cp_async16_if(void *dst, const void *src, bool live) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-                 "r"(live ? 16 : 0)
-                 : "memory");
-}
-
-__device__ __forceinline__ int xchunk(int c) { return c ^ (((c >> 3) & 1) << 1); }
-
-// D += A * B, m16n8k16 bf16 -> fp32, as a pure function of its operands (not
-// volatile), so that the compiler may interleave independent items.
-__device__ __forceinline__ void mma_pure(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 
 
 template <int MX, int NT, bool BLK>
@@ -198,17 +162,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
     // item (group j of this warp, tile k) into ring slot s
     // (items past the end copy nothing: a source size of 0 writes zeros, and
     // the address stays in bounds)
-    auto issue = [&](int j, int k, int s) {
+    auto issue = [&](int j, int k, uint8_t *dst) {
         const bool live = j < gpw && (k + 1 < NT || full);
         const uint32_t *src = qbase + min(j, gpw - 1) * (kWarps * 16);
-        cp_async16_if(ring + s * (2 * kThreads * 16), src + off0[k], live);
-        cp_async16_if(ring + s * (2 * kThreads * 16) + kThreads * 16, src + off1[k], live);
+        cp_async16_if(dst, src + off0[k], live);
+        cp_async16_if(dst + kThreads * 16, src + off1[k], live);
         cp_async_commit();
     };
 #pragma unroll
     for (int d = 0; d < D; ++d)
 #pragma unroll
-        for (int k = 0; k < NT; ++k) issue(d, k, d * NT + k);
+        for (int k = 0; k < NT; ++k) issue(d, k, ring + (d * NT + k) * (2 * kThreads * 16));
     pdl_launch_dependents();
     if (threadIdx.x == 0) {
         l2_prefetch_share(p.pf, blockIdx.x, gridDim.x);
@@ -304,12 +268,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
     for (int n8 = 0; n8 < NTOK; ++n8)
 #pragma unroll
         for (int i = 0; i < 16; ++i) xb[n8][i] = 0u;
+    // one group per iteration, not unrolled over the ring's D groups (a
+    // smaller loop body: fewer instruction-cache misses), with the group's
+    // ring slots found from d = j mod D at run time
 #pragma unroll 1
-    for (int j0 = 0; j0 < gpw; j0 += D) {
-#pragma unroll
-        for (int d = 0; d < D; ++d) {
-            const int j = j0 + d;
-            if (j < gpw) {
+    for (int j = 0, d = 0; j < gpw; ++j, d = d + 1 == D ? 0 : d + 1) {
+        uint8_t *const slots = ring + d * (NT * 2 * kThreads * 16);
+        {
+            {
                 const int gi = warp + kWarps * j;
 #pragma unroll
                 for (int n8 = 0; n8 < NTOK; ++n8) {
@@ -392,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
                 };
                 // one item: tile k of group gi, from ring slot d * NT + k
                 auto item = [&](int k) {
-                    const uint8_t *src = ring + (d * NT + k) * (2 * kThreads * 16);
+                    const uint8_t *src = slots + k * (2 * kThreads * 16);
                     const uint4 wa = *reinterpret_cast<const uint4 *>(src);
                     const uint4 wb = *reinterpret_cast<const uint4 *>(src + kThreads * 16);
                     const uint32_t sz0 = szs[(k * 16 + g) * SZS + gi];
@@ -425,12 +391,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
                         cp_async_wait_group<R - 2>();
                         item(k);
                         if (k + 2 < NT || full) item(k + 1);
-                        issue(j + D, k, d * NT + k);
-                        issue(j + D, k + 1, d * NT + k + 1);
+                        issue(j + D, k, slots + k * (2 * kThreads * 16));
+                        issue(j + D, k + 1, slots + (k + 1) * (2 * kThreads * 16));
                     } else {
                         cp_async_wait_group<R - 1>();
                         if (full) item(k);
-                        issue(j + D, k, d * NT + k);
+                        issue(j + D, k, slots + k * (2 * kThreads * 16));
                     }
                 }
             }
@@ -623,6 +589,10 @@ mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y
     p.pf = pf;
     const StreamLayout L(M, p.K, p.Gp, p.csr_cap, nt, p.blk_cap, p.blk_words);
     if (L.total > kMaxSmem) return MQ_ERR_UNSUPPORTED;
+    // one CTA per SM (X takes the shared memory of two) and more CTAs than
+    // SMs: a second wave; the tall-layer kernel, which reads X from L2, or
+    // the register kernels take the call
+    if (L.total > kTwoPerSm && grid > sm_count()) return MQ_ERR_UNSUPPORTED;
     const int mx = M == 1 ? 0 : M <= 8 ? 1 : 2;
     void *kern = use_blocks ? (mx == 0 ? kernel_for<1, true>(nt) : mx == 1 ? kernel_for<8, true>(nt)
                                                                          : kernel_for<16, true>(nt))

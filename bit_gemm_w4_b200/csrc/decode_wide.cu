@@ -105,14 +105,6 @@ constexpr int kFrag = 512;               // 16 rows x 16 k-slots of bf16, A-frag
 constexpr int kTileBytes = 4 * kFrag;    // the fragments of four k-steps
 __host__ __device__ constexpr int ring_offset(int spr) { return wtab_bytes(spr) + kWarps * kTileBytes; }
 
-// Byte offset in a fragment tile of the code at row r (0..15), column c of a
-// 128-column group: thread (g = r % 8, t = c / 32) holds it in register
-// (r / 8) + 2 * ((c % 4) / 2), half c % 2 (the m16n8k16 A layout under the
-// packed codes' k order, where k-step (c % 32) / 4 covers column c).
-__device__ __forceinline__ int tile_pos(int r, int c) {
-    return (((r & 7) * 4 + (c >> 5)) * 4 + (r >> 3) + 2 * ((c & 3) >> 1)) * 4 + (c & 1) * 2;
-}
-
 // The same for the int8 m16n8k32 A layout (W4A4): column c of a group sits
 // at byte ((c & 3) << 1) | ((c >> 2) & 1) of its 8-column chunk in the
 // packed codes' k order; positions 0..3 go to registers (r / 8), 4..7 to
@@ -121,8 +113,6 @@ __device__ __forceinline__ int tile_pos_a4(int r, int c) {
     const int pos = ((c & 3) << 1) | ((c >> 2) & 1);
     return ((r & 7) * 4 + (c >> 5)) * 16 + ((r >> 3) + ((pos >> 2) << 1)) * 4 + (pos & 3);
 }
-
-__device__ __forceinline__ int xchunk(int c) { return c ^ (((c >> 3) & 1) << 1); }
 
 template <bool A4, int NS>
 __global__ void __launch_bounds__(kThreads, 2)

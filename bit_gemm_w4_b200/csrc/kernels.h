@@ -45,6 +45,15 @@ struct DeviceWeight {
     const uint16_t *wide_off;  // [ceil(N/128) * S * kWideOffStride]
     const uint16_t *wide_ent;  // [nnz] (+ padding)
     int64_t wide_max;          // longest slice, entries
+    // The residual again, grouped for the tall-layer decode kernel: per
+    // (16-row tile, 128-column group, half-group) key (tile * G + group) * 2
+    // + (column % 32) / 16 a list of u16 entries, in CSR order inside a key:
+    // the byte offset of the code in the half-group's four 512-byte m16n8k16
+    // A-fragment tiles (11 bits: k-step % 4 * 512 + the fragment position of
+    // (row % 16, column % 128)) | (q_r & 0xF) << 11. tl_ptr[key] is the first
+    // entry of a key (one more at the end). NULL when nnz = 0.
+    const int32_t *tl_ptr;     // [ceil(N/16) * G * 2 + 1]
+    const uint16_t *tl_ent;    // [nnz] (+ padding)
     // The residual again as block tiles, when it consists of whole 16 x 64
     // blocks (block allocation; NULL otherwise): per 16-row block-row the
     // offsets of its blocks, their column-block indices, 512 bytes of
@@ -113,6 +122,17 @@ mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaS
 mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y,
                                cudaStream_t stream, float *partial = nullptr,
                                const L2Prefetch &pf = L2Prefetch());
+
+// Tall-layer decode kernel (decode_tall.cu) for 2 <= M <= 16 on layers of
+// at least four 16-row tiles per CTA at two CTAs per SM: X from L2, a
+// per-thread item ring, the residual as tensor-core k-steps from the
+// per-tile lists (DeviceWeight::tl_ptr). `partial` and `pf` as for
+// launch_decode. Returns MQ_ERR_UNSUPPORTED (without setting an error
+// message) for other layers or when a CTA's lists or scale words do not fit
+// its shared memory.
+mq_status launch_decode_tall(const mq_weight *w, const void *X, int M, void *Y,
+                             cudaStream_t stream, float *partial = nullptr,
+                             const L2Prefetch &pf = L2Prefetch());
 
 // Wide decode kernel (decode_wide.cu) for 8 < M <= 16; `partial` as for
 // decode. Returns MQ_ERR_UNSUPPORTED (without setting an error message) when

@@ -76,6 +76,7 @@ def _load():
         "mq_pack_host": ([vp, i64, i64, ctypes.POINTER(_PackOpts), ctypes.POINTER(_HostPacked)], st),
         "mq_prefill_lists_host": ([i64, i64, vp, vp, vp, vp, vp], st),
         "mq_wide_lists_host": ([i64, i64, vp, vp, vp, vp, vp, vp, ctypes.POINTER(i64)], st),
+        "mq_tile_lists_host": ([i64, i64, vp, vp, vp, vp, vp], st),
         "mq_pack_decomposed": ([ctypes.POINTER(_Decomp), vp, ctypes.POINTER(vp)], st),
         "mq_get_info": ([vp, ctypes.POINTER(_Info)], st),
         "mq_export": ([vp, ctypes.POINTER(_HostPacked)], st),
@@ -189,6 +190,20 @@ def wide_lists_host(N: int, K: int, packed: dict):
     _check(_lib.mq_wide_lists_host(N, K, _ptr(row_ptr), _ptr(col), _ptr(val), _ptr(ptr), _ptr(off),
                                    _ptr(ent), ctypes.byref(mx)), "mq_wide_lists_host")
     return ptr, off, ent[:nnz], int(mx.value)
+
+
+def tile_lists_host(N: int, K: int, packed: dict):
+    """The tall-layer decode kernel's residual lists of a host pack: (ptr
+    int32 [ceil(N/16) * K/128 * 2 + 1], ent uint16 [nnz]); no CUDA call."""
+    row_ptr = np.ascontiguousarray(packed["row_ptr"], np.int32)
+    col = np.ascontiguousarray(packed["col"], np.uint16)
+    val = np.ascontiguousarray(packed["val"], np.uint8)
+    nnz = int(row_ptr[-1])
+    ptr = np.zeros(((N + 15) // 16) * (K // 128) * 2 + 1, np.int32)
+    ent = np.zeros(max(nnz, 1), np.uint16)
+    _check(_lib.mq_tile_lists_host(N, K, _ptr(row_ptr), _ptr(col), _ptr(val), _ptr(ptr), _ptr(ent)),
+           "mq_tile_lists_host")
+    return ptr, ent[:nnz]
 
 
 def selftest_bounded_wait(limit_cycles: int = 1 << 20) -> list:

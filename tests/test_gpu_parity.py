@@ -391,6 +391,32 @@ def test_tall_layer_decode(mq, cuda, M, K, rho):
     assert ru["ok"], ru
 
 
+@pytest.mark.parametrize("rho", [0.01, 0.04])
+def test_tall_kernel_sampled_rows(mq, cuda, rho):
+    # 2-16 tokens on a layer tall enough for the tall-layer kernel (19000
+    # rows, the last 16-row tile ragged) whose X (K = 8192) does not fit the
+    # streaming kernel's shared memory; at rho = 4 % a CTA's residual lists
+    # exceed their budget and the wide and register kernels take the call.
+    # Fused and unfused, checked on sampled rows.
+    N, K = 19000, 8192
+    W = synth.weight(N, K, std=0.015, outlier_frac=0.01, outlier_cols=32, seed=71)
+    w = mq.Weight.pack(W, rho)
+    rows = np.unique(np.concatenate([np.arange(0, 40), np.arange(N - 24, N),
+                                     np.random.default_rng(1).choice(N, 64, replace=False)]))
+    d = oracle.decompose(np.ascontiguousarray(W[rows]), rho)
+    del W
+    for M in (2, 5, 8, 12, 16):
+        X = synth.activations(M, K, seed=72 + M, channels=4, mult=20.0)
+        Y = w.linear(X.cuda())
+        Yu = w.linear_unfused(X.cuda())
+        torch.cuda.synchronize()
+        assert w.device_error() == 0
+        r = oracle_check(Y[:, rows], X, d)
+        assert r["ok"], (M, r)
+        r = oracle_check(Yu[:, rows], X, d)
+        assert r["ok"], (M, "unfused", r)
+
+
 @pytest.mark.parametrize("M", [17, 40])
 def test_longest_k_prefill(mq, cuda, M):
     # K = 65536 at more than 16 tokens: the prefill kernel reads 512 scale

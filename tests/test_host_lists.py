@@ -109,3 +109,58 @@ def test_wide_lists_regroup_the_csr(N, K, rho, blocks):
     assert np.array_equal(off[:, :129].astype(np.int64), eoff[:, :129])
     assert np.array_equal(ent.astype(np.int64), eent)
     assert mx == int(np.diff(eptr).max(initial=0))
+
+
+def _fragment_byte(r, c):
+    """Byte of the code at (row r, column c) of a 16-row x 128-column group in
+    the m16n8k16 bf16 A fragments of its k-step, from the fragment's
+    definition: thread 4 * (row % 8) + kk % 8 / 2 holds element (row, kk) in
+    register (row >= 8) + 2 * (kk >= 8), half kk % 2; under the packed
+    codes' nibble interleave, k-step s of thread t covers columns 32t + 4s +
+    {0, 1} as kk = 2t + {0, 1} and 32t + 4s + {2, 3} as kk = 2t + 8 + {0, 1}."""
+    t, s, j = c // 32, (c % 32) // 4, c % 4
+    kk = 2 * t + (j % 2) + (8 if j >= 2 else 0)
+    lane = 4 * (r % 8) + (kk % 8) // 2
+    reg = int(r >= 8) + 2 * int(kk >= 8)
+    return (s % 4) * 512 + lane * 16 + reg * 4 + (kk % 2) * 2
+
+
+def _tile_expected(N, K, packed):
+    G = K // 128
+    keys = ((N + 15) // 16) * G * 2
+    buckets = [[] for _ in range(keys)]
+    rp, col, val = packed["row_ptr"], packed["col"], packed["val"]
+    for n in range(N):
+        for e in range(rp[n], rp[n + 1]):
+            c = int(col[e])
+            nib = (int(val[e >> 1]) >> ((e & 1) * 4)) & 0xF
+            key = ((n // 16) * G + c // 128) * 2 + (c % 32) // 16
+            buckets[key].append(_fragment_byte(n % 16, c % 128) | (nib << 11))
+    ptr = np.zeros(keys + 1, np.int64)
+    for k in range(keys):
+        ptr[k + 1] = ptr[k] + len(buckets[k])
+    return ptr, np.array([w for b in buckets for w in b], np.int64)
+
+
+@pytest.mark.parametrize("N,K,rho,blocks", [
+    (300, 640, 0.05, None),      # ragged last tile, five groups
+    (256, 1024, 0.0, 0.25),      # block mode
+    (128, 256, 0.0, None),       # no residual
+])
+def test_tile_lists_regroup_the_csr(N, K, rho, blocks):
+    W = synth.weight(N, K, std=0.02, outlier_frac=0.01, seed=3 * N + K)
+    packed = mq.pack_host(W, rho, block_fraction=blocks)
+    ptr, ent = mq.tile_lists_host(N, K, packed)
+    eptr, eent = _tile_expected(N, K, packed)
+    assert np.array_equal(ptr.astype(np.int64), eptr)
+    assert np.array_equal(ent.astype(np.int64), eent)
+
+
+def test_fragment_byte_covers_each_k_step_once():
+    # every (row, column) of a half-group's four k-steps lands on its own byte
+    # pair, and the sixteen rows x sixteen columns of one k-step fill its 512
+    # bytes exactly
+    for h in (0, 1):
+        cols = [c for c in range(128) if (c % 32) // 16 == h]
+        seen = {_fragment_byte(r, c) for r in range(16) for c in cols}
+        assert len(seen) == 16 * len(cols) and seen == set(range(0, 2048, 2))
