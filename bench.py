@@ -69,8 +69,13 @@ def alg_bytes(M: int, N: int, K: int, nnz: int) -> int:
 # 7B shape (M = 1, density 0.5 %), each from one ncu capture of that shape
 # (profiles/decode_stream_kernel_7b_m1.txt gives the commands). Set to None
 # when the kernel changes until it is captured again.
-DECODE_TRAFFIC = {(4096, 4096): 9.223168e6, (11008, 4096): 24.663808e6,
-                  (4096, 11008): 24.668928e6}
+DECODE_TRAFFIC = {(4096, 4096): 9.193728e6, (11008, 4096): 24.641024e6,
+                  (4096, 11008): 24.639488e6}
+
+# DRAM bytes (read + write) of one launch of the tall-layer decode kernel on
+# the 70B MLP shape (M = 16, density 1 %), from one ncu capture
+# (profiles/decode_tall_kernel_70b_m16.txt). None when the kernel changes.
+TALL_TRAFFIC = 131.396864e6 + 6.799616e6
 
 
 def alg_flops(M: int, N: int, K: int, nnz: int) -> int:
@@ -474,13 +479,13 @@ def secondary(torch, mq, dev, stream, pk, which: str, reps: int):
     """One secondary workload, device time per launch.
 
     Decode (the 70B MLP at M = 16): back-to-back launches replayed from a
-    CUDA graph, alternating between two packed copies of the weight (264 MB,
-    twice the L2), as the primary line times its step. Prefill: single
+    CUDA graph, rotating over three packed copies of the weight (396 MB, a
+    copy's reuse distance twice the L2), as the primary line times its step. Prefill: single
     launches after an L2 flush (median of `reps`); each launch re-reads its
     weight per token tile, so L2 matters little there."""
     from bit_gemm_w4_b200 import synth
     decode = which != "prefill"
-    copies = 2 if decode else 1
+    copies = 3 if decode else 1
     ds = DecodeSet(mq, torch, which, copies, dev)
     N, K = ds.shapes[0]
     for c in range(copies):
@@ -522,6 +527,7 @@ def secondary(torch, mq, dev, stream, pk, which: str, reps: int):
         del flush
     by, fl = ds.bytes_per_launch[0], ds.flops_per_launch[0]
     out = {"workload": which, "M": ds.M, "N": N, "K": K, "nnz": ds.nnz[0], "ms": ms,
+           "kernel": "decode_tall_kernel" if decode else "prefill_kernel",
            "TB_s": by / ms / 1e9, "TFLOP_s": fl / ms / 1e9, "timing": timing}
     if which == "prefill":
         peak = pk["bf16_tflops"]
@@ -530,7 +536,8 @@ def secondary(torch, mq, dev, stream, pk, which: str, reps: int):
     else:
         peak = pk["hbm_gbs"]
         out["roofline"] = {"bound": "hbm", "achieved": by / ms / 1e6, "peak": peak,
-                           "unit": "GB/s", "frac": by / ms / 1e6 / peak}
+                           "unit": "GB/s", "frac": by / ms / 1e6 / peak,
+                           "traffic": TALL_TRAFFIC}
     del ds
     return out
 
