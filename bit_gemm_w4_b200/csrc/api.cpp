@@ -160,17 +160,16 @@ void build_wide_lists(const HostPacked &hp, std::vector<int32_t> &ptr, std::vect
         }
 }
 
-// The residual grouped per (16-row tile, 128-column group, half-group) for
-// the tall-layer decode kernel (layout in kernels.h, DeviceWeight::tl_ptr).
-// The half-group of column c is (c % 32) / 16: under the nibble interleave,
-// MMA k-step (c % 32) / 4 covers c, so each half holds four of the group's
-// eight k-steps. An entry is stored as the byte where its code goes in the
-// half's four m16n8k16 A-fragment tiles (512 bytes each; inside one, thread
-// (g = r % 8, t = c / 32) holds it in register (r / 8) + 2 * ((c % 4) / 2),
-// half c % 2), with the stored nibble above it.
+// The residual grouped per (16-row tile, 128-column group) for the
+// tall-layer decode kernel (layout in kernels.h, DeviceWeight::tl_ptr). An
+// entry is stored as the byte where its code goes in the group's eight
+// m16n8k16 A-fragment tiles (512 bytes each, one per MMA k-step; under the
+// nibble interleave k-step (c % 32) / 4 covers column c, and inside a tile
+// thread (g = r % 8, t = c / 32) holds it in register (r / 8) + 2 * ((c % 4)
+// / 2), half c % 2), with the stored nibble above it.
 void build_tile_lists(const HostPacked &hp, std::vector<int32_t> &ptr, std::vector<uint16_t> &ent) {
-    const int64_t tiles = (hp.N + 15) / 16, G = hp.K / 128, keys = tiles * G * 2;
-    auto key = [&](int64_t n, int64_t c) { return ((n / 16) * G + c / 128) * 2 + (c % 32) / 16; };
+    const int64_t tiles = (hp.N + 15) / 16, G = hp.K / 128, keys = tiles * G;
+    auto key = [&](int64_t n, int64_t c) { return (n / 16) * G + c / 128; };
     ptr.assign(static_cast<size_t>(keys + 1), 0);
     for (int64_t n = 0; n < hp.N; ++n)
         for (int64_t e = hp.row_ptr[n]; e < hp.row_ptr[n + 1]; ++e) ++ptr[key(n, hp.col[e]) + 1];
@@ -182,9 +181,9 @@ void build_tile_lists(const HostPacked &hp, std::vector<int32_t> &ptr, std::vect
             const int64_t c = hp.col[e];
             const uint32_t nib = (hp.val[e >> 1] >> ((e & 1) * 4)) & 0xF;
             const int64_t r = n % 16, cg = c % 128;
-            const int64_t pos = ((cg % 32) / 4 % 4) * 512 +
+            const int64_t pos = ((cg % 32) / 4) * 512 +
                                 (((r % 8) * 4 + cg / 32) * 4 + r / 8 + 2 * ((cg % 4) / 2)) * 4 + (cg % 2) * 2;
-            ent[fill[key(n, c)]++] = static_cast<uint16_t>(pos | (nib << 11));
+            ent[fill[key(n, c)]++] = static_cast<uint16_t>(pos | (nib << 12));
         }
 }
 

@@ -26,12 +26,12 @@
 //     of 128.0, then a subtraction of 128 + z), mma.sync m16n8k16 in fp32 for
 //     one or two 8-token column tiles, the group partial scaled by s in fp32.
 //   * Residual, per item, on the tensor cores: the host groups the residual
-//     per (tile, group, half-group) (DeviceWeight::tl_ptr), each entry
-//     carrying its byte in the A fragments; the CTA stages its run's lists
-//     once. For each half-group holding entries, the warp's lanes scatter them
-//     as exact bf16 codes into four zeroed 512-byte fragment tiles, and each
-//     k-step that received an entry costs one more mma.sync per token tile on
-//     the X fragment already in registers; the sums are scaled by the row's
+//     per (tile, group) (DeviceWeight::tl_ptr), each entry carrying its byte
+//     in the A fragments; the CTA stages its run's lists once. The warp's
+//     lanes scatter an item's entries as exact bf16 codes into eight zeroed
+//     512-byte fragment tiles, and each k-step that received an entry costs
+//     one more mma.sync per token tile on the X fragment already in
+//     registers; the sums are scaled by the row's
 //     s_r and added in. The residual runs after the group's dense items, in
 //     a loop over the tiles that is not unrolled (the unrolled form outgrew
 //     the instruction cache).
@@ -59,7 +59,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kTMin = 4;                   // fewest tiles per CTA (X is read once per CTA and group)
 constexpr int kTMax = 8;                   // most tiles per CTA (one accumulator set each)
 constexpr int kSlotBytes = 2 * kThreads * 16;  // one item: 16 bytes of rows g and g + 8 per thread
-constexpr int kFragBytes = 4 * 512;        // per warp: the A fragments of four k-steps
+constexpr int kFragBytes = 8 * 512;        // per warp: the A fragments of a group's eight k-steps
 constexpr int kTwoPerSm = 113 * 1024;      // shared memory of each of two CTAs per SM
 constexpr int kEntBudget = 24 * 1024;      // shared memory for a CTA's residual entries
 
@@ -87,6 +87,13 @@ struct TallParams {
 // its X fragment.
 __host__ __device__ constexpr int group_lanes(int mx) { return mx > 8 ? kWarps / 2 : kWarps; }
 
+// Scale/zero rows in shared memory: with Gp a multiple of 32, Gp words per
+// row and 16-byte chunk q of row r stored at chunk q ^ (r % 8), so that the
+// eight rows a warp reads at once (g = 0..7) fall on distinct banks; else the
+// rows are padded to an odd multiple of four words.
+__host__ __device__ inline bool sz_swizzled(int Gp) { return Gp % 32 == 0; }
+__host__ __device__ inline int tall_sz_stride(int Gp) { return sz_swizzled(Gp) ? Gp : sz_stride(Gp); }
+
 // Shared-memory layout (bytes), identical on host and device. After the
 // dense pass the reduction buffer [GL][NT][M][16] fp32 reuses it from 0.
 struct TallLayout {
@@ -94,11 +101,11 @@ struct TallLayout {
     __host__ __device__ TallLayout(int M, int G, int Gp, int nt, int R, int ent_cap) {
         const bool resid = ent_cap > 0;
         ring = 0;                                               // [R][2][kThreads][16 B]
-        szs = ring + R * kSlotBytes;                            // [NT * 16][sz_stride] words
-        toff = szs + nt * 16 * sz_stride(Gp) * 4;               // [NT * G * 2 + 1] u16
-        tent = toff + (resid ? ((nt * G * 2 + 1) * 2 + 15) / 16 * 16 : 0);
+        szs = ring + R * kSlotBytes;                            // [NT * 16][tall_sz_stride] words
+        toff = szs + nt * 16 * tall_sz_stride(Gp) * 4;          // [NT * G + 1] u16
+        tent = toff + (resid ? ((nt * G + 1) * 2 + 15) / 16 * 16 : 0);
         frag = tent + (resid ? ((ent_cap + 8) * 2 + 15) / 16 * 16 : 0);  // from a 16-byte aligned start
-        rsf = frag + (resid ? kWarps * kFragBytes : 0);          // [kWarps][4][512 B]
+        rsf = frag + (resid ? kWarps * kFragBytes : 0);          // [kWarps][8][512 B]
         total = rsf + (resid ? nt * 16 * 4 : 0);                 // [NT * 16] fp32 s_r
         const int red = group_lanes(M) * nt * M * 16 * 4;
         if (total < red) total = red;
@@ -116,7 +123,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tall_kernel(const __grid_c
     const int g = lane >> 2, t = lane & 3;
     const int M = p.M, N = p.N, K = p.K, G = p.G;
     const TallLayout L(M, G, p.Gp, NT, R, p.ent_cap);
-    const int SZS = sz_stride(p.Gp);
+    const int SZS = tall_sz_stride(p.Gp);
+    const bool swz = sz_swizzled(p.Gp);
     const int t0 = static_cast<int>(static_cast<long long>(p.ntile) * blockIdx.x / gridDim.x);
     const int t1 = static_cast<int>(static_cast<long long>(p.ntile) * (blockIdx.x + 1) / gridDim.x);
     const int nt = t1 - t0;  // NT or NT - 1
@@ -134,12 +142,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tall_kernel(const __grid_c
         const int q4 = p.Gp / 4;  // 16-byte chunks per scale/zero row
         for (int i = threadIdx.x; i < (n_hi - n_lo) * q4; i += kThreads) {
             const int r = i / q4, q = i - r * q4;
-            cp_async16(smem + L.szs + (r * SZS + 4 * q) * 4,
+            cp_async16(smem + L.szs + (r * SZS + 4 * (swz ? q ^ (r & 7) : q)) * 4,
                        p.sz + static_cast<size_t>(n_lo + r) * p.Gp + 4 * q);
         }
     }
     if (resid) {
-        const int k_lo = t0 * G * 2, k_hi = k_lo + nt * G * 2;
+        const int k_lo = t0 * G, k_hi = k_lo + nt * G;
         const int e_lo = p.tl_ptr[k_lo], e_hi = p.tl_ptr[k_hi];
         const int e_base = e_lo & ~7;
         const int n16 = ((e_hi - e_base) * 2 + 15) / 16;
@@ -184,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tall_kernel(const __grid_c
     __syncthreads();
 
     const uint32_t *szw = reinterpret_cast<const uint32_t *>(smem + L.szs) + (kt0 * 16 + g) * SZS;
-    const uint16_t *tow = reinterpret_cast<const uint16_t *>(smem + L.toff) + kt0 * G * 2;
+    const uint16_t *tow = reinterpret_cast<const uint16_t *>(smem + L.toff) + kt0 * G;
     const uint16_t *tent = reinterpret_cast<const uint16_t *>(smem + L.tent);
     const float *rsw = reinterpret_cast<const float *>(smem + L.rsf) + kt0 * 16 + g;
     uint8_t *const frag = smem + L.frag + warp * kFragBytes;
@@ -206,6 +214,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tall_kernel(const __grid_c
 #pragma unroll 1
     for (int j = 0; j < gpw; ++j, base = (base + NTW) & (R - 1)) {
         const int gi = gl + GL * j;
+        // the group's word in this thread's scale/zero rows (g and g + 8 of
+        // each tile: both r % 8 = g under the swizzle)
+        const int gis = swz ? ((((gi >> 2) ^ g) << 2) | (gi & 3)) : gi;
         // X fragment of the group for tokens g and g + 8: columns 32t .. 32t + 31
 #pragma unroll
         for (int n8 = 0; n8 < NTOK; ++n8) {
@@ -235,42 +246,49 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tall_kernel(const __grid_c
             }
         };
         // the residual code sums rc of tile k (a run-time index) in group gi:
-        // per half-group with entries, scatter the codes into the fragment
-        // tiles (each entry carries its byte there), one MMA per token tile
-        // for each k-step that received one, the lanes clearing their
-        // fragment after reading it; false when the item has no entries
+        // scatter the item's entries into the fragment tiles of the group's
+        // eight k-steps (each entry carries its byte there), then one MMA per
+        // token tile for each k-step that received one (two accumulator chains
+        // at one token tile), the lanes clearing their fragment after reading
+        // it; false when the item has no entries
         auto residual = [&](int k, float (&rc)[NTOK][4]) {
-            const uint16_t *to = tow + (k * G + gi) * 2;
-            const int e0 = to[0], e1 = to[1], e2 = to[2];
-            if (e2 == e0) return false;  // the same for every lane
+            const uint16_t *to = tow + k * G + gi;
+            const int e0 = to[0], e1 = to[1];
+            if (e1 == e0) return false;  // the same for every lane
+            uint32_t used = 0;  // k-steps that received an entry
+            for (int e = e0 + lane; e < e1; e += 32) {
+                const uint32_t v = tent[e];
+                const uint32_t pos = v & 0xFFFu;
+                const int q = static_cast<int>((v >> 12) ^ 8u) - 8;
+                sts_u16(frag + pos, __float_as_uint(static_cast<float>(q)) >> 16);
+                used |= 1u << (pos >> 9);
+            }
+            used = __reduce_or_sync(0xffffffffu, used);
+            __syncwarp();
+            float rd[NTOK][4];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int lo = h ? e1 : e0, hi = h ? e2 : e1;
-                if (hi > lo) {
-                    uint32_t used = 0;  // k-steps of the half that received an entry
-                    for (int e = lo + lane; e < hi; e += 32) {
-                        const uint32_t v = tent[e];
-                        const uint32_t pos = v & 0x7FFu;
-                        const int q = static_cast<int>((v >> 11) ^ 8u) - 8;
-                        sts_u16(frag + pos, __float_as_uint(static_cast<float>(q)) >> 16);
-                        used |= 1u << (pos >> 9);
+            for (int n8 = 0; n8 < NTOK; ++n8)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) rd[n8][i] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                if ((used >> ks) & 1u) {
+                    const uint4 f = lds128(frag + ks * 512 + 16 * lane);
+                    sts128(frag + ks * 512 + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
+                    const uint32_t fa[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                    for (int n8 = 0; n8 < NTOK; ++n8) {
+                        if (NTOK == 1 && (ks & 1))
+                            mma_pure(rd[n8], fa, xb[n8][2 * ks], xb[n8][2 * ks + 1]);
+                        else
+                            mma_pure(rc[n8], fa, xb[n8][2 * ks], xb[n8][2 * ks + 1]);
                     }
-                    used = __reduce_or_sync(0xffffffffu, used);
-                    __syncwarp();
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        if ((used >> u) & 1u) {
-                            const uint4 f = lds128(frag + u * 512 + 16 * lane);
-                            sts128(frag + u * 512 + 16 * lane, make_uint4(0u, 0u, 0u, 0u));
-                            const uint32_t fa[4] = {f.x, f.y, f.z, f.w};
-                            const int ks = 4 * h + u;
-#pragma unroll
-                            for (int n8 = 0; n8 < NTOK; ++n8)
-                                mma_pure(rc[n8], fa, xb[n8][2 * ks], xb[n8][2 * ks + 1]);
-                        }
-                    }
-                    __syncwarp();
                 }
+            }
+            __syncwarp();
+            if (NTOK == 1) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) rc[0][i] += rd[0][i];
             }
             return true;
         };
@@ -279,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tall_kernel(const __grid_c
             const uint8_t *src = slot(k);
             const uint4 wa = *reinterpret_cast<const uint4 *>(src);
             const uint4 wb = *reinterpret_cast<const uint4 *>(src + kThreads * 16);
-            const uint32_t sz0 = szw[k * 16 * SZS + gi];
-            const uint32_t sz1 = szw[(k * 16 + 8) * SZS + gi];
+            const uint32_t sz0 = szw[k * 16 * SZS + gis];
+            const uint32_t sz1 = szw[(k * 16 + 8) * SZS + gis];
             const uint32_t zz0 = zero_pair(sz0), zz1 = zero_pair(sz1);
             const uint32_t bias = p.bias;
             // one accumulator chain per token tile

@@ -46,13 +46,13 @@ struct DeviceWeight {
     const uint16_t *wide_ent;  // [nnz] (+ padding)
     int64_t wide_max;          // longest slice, entries
     // The residual again, grouped for the tall-layer decode kernel: per
-    // (16-row tile, 128-column group, half-group) key (tile * G + group) * 2
-    // + (column % 32) / 16 a list of u16 entries, in CSR order inside a key:
-    // the byte offset of the code in the half-group's four 512-byte m16n8k16
-    // A-fragment tiles (11 bits: k-step % 4 * 512 + the fragment position of
-    // (row % 16, column % 128)) | (q_r & 0xF) << 11. tl_ptr[key] is the first
-    // entry of a key (one more at the end). NULL when nnz = 0.
-    const int32_t *tl_ptr;     // [ceil(N/16) * G * 2 + 1]
+    // (16-row tile, 128-column group) key tile * G + group a list of u16
+    // entries, in CSR order inside a key: the byte offset of the code in the
+    // group's eight 512-byte m16n8k16 A-fragment tiles (12 bits: k-step * 512
+    // + the fragment position of (row % 16, column % 128)) | (q_r & 0xF) << 12.
+    // tl_ptr[key] is the first entry of a key (one more at the end). NULL
+    // when nnz = 0.
+    const int32_t *tl_ptr;     // [ceil(N/16) * G + 1]
     const uint16_t *tl_ent;    // [nnz] (+ padding)
     // The residual again as block tiles, when it consists of whole 16 x 64
     // blocks (block allocation; NULL otherwise): per 16-row block-row the

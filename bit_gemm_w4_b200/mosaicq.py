@@ -194,12 +194,12 @@ def wide_lists_host(N: int, K: int, packed: dict):
 
 def tile_lists_host(N: int, K: int, packed: dict):
     """The tall-layer decode kernel's residual lists of a host pack: (ptr
-    int32 [ceil(N/16) * K/128 * 2 + 1], ent uint16 [nnz]); no CUDA call."""
+    int32 [ceil(N/16) * K/128 + 1], ent uint16 [nnz]); no CUDA call."""
     row_ptr = np.ascontiguousarray(packed["row_ptr"], np.int32)
     col = np.ascontiguousarray(packed["col"], np.uint16)
     val = np.ascontiguousarray(packed["val"], np.uint8)
     nnz = int(row_ptr[-1])
-    ptr = np.zeros(((N + 15) // 16) * (K // 128) * 2 + 1, np.int32)
+    ptr = np.zeros(((N + 15) // 16) * (K // 128) + 1, np.int32)
     ent = np.zeros(max(nnz, 1), np.uint16)
     _check(_lib.mq_tile_lists_host(N, K, _ptr(row_ptr), _ptr(col), _ptr(val), _ptr(ptr), _ptr(ent)),
            "mq_tile_lists_host")

@@ -312,16 +312,15 @@ mq_status mq_wide_lists_host(int64_t N, int64_t K, const int32_t *row_ptr, const
                              int64_t *max_len);
 
 /* Test support, no CUDA call: the residual of a host pack regrouped as the
- * tall-layer decode kernel reads it, per key (row / 16 * (K/128) + column /
- * 128) * 2 + (column % 32) / 16 (16-row tile, 128-column group, half of the
- * group's eight MMA k-steps), K a multiple of 128. Each entry is stored as
- * the byte it takes in the half's four m16n8k16 bf16 A-fragment tiles (512
- * bytes per k-step; k-step (column % 32) / 4, where under the packed codes'
- * nibble interleave thread t = (column % 128) / 32 of row group row % 8 holds
- * it in register row % 16 / 8 + 2 * ((column % 4) / 2), half column % 2):
- * ((column % 32) / 4 % 4) * 512 + ((row % 8) * 4 + t) * 16 + register * 4 +
- * half * 2, with the stored nibble << 11. Writes ptr: int32
- * [ceil(N/16) * (K/128) * 2 + 1] key starts; ent: uint16 [nnz] in CSR order
+ * tall-layer decode kernel reads it, per key row / 16 * (K/128) + column /
+ * 128 (16-row tile, 128-column group), K a multiple of 128. Each entry is
+ * stored as the byte it takes in the group's eight m16n8k16 bf16 A-fragment
+ * tiles (512 bytes per MMA k-step; k-step (column % 32) / 4, where under the
+ * packed codes' nibble interleave thread t = (column % 128) / 32 of row group
+ * row % 8 holds it in register row % 16 / 8 + 2 * ((column % 4) / 2), half
+ * column % 2): ((column % 32) / 4) * 512 + ((row % 8) * 4 + t) * 16 +
+ * register * 4 + half * 2, with the stored nibble << 12. Writes ptr: int32
+ * [ceil(N/16) * (K/128) + 1] key starts; ent: uint16 [nnz] in CSR order
  * inside a key. Errors as mq_prefill_lists_host. */
 mq_status mq_tile_lists_host(int64_t N, int64_t K, const int32_t *row_ptr, const uint16_t *col,
                              const uint8_t *val, int32_t *ptr, uint16_t *ent);

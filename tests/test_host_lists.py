@@ -122,20 +122,20 @@ def _fragment_byte(r, c):
     kk = 2 * t + (j % 2) + (8 if j >= 2 else 0)
     lane = 4 * (r % 8) + (kk % 8) // 2
     reg = int(r >= 8) + 2 * int(kk >= 8)
-    return (s % 4) * 512 + lane * 16 + reg * 4 + (kk % 2) * 2
+    return s * 512 + lane * 16 + reg * 4 + (kk % 2) * 2
 
 
 def _tile_expected(N, K, packed):
     G = K // 128
-    keys = ((N + 15) // 16) * G * 2
+    keys = ((N + 15) // 16) * G
     buckets = [[] for _ in range(keys)]
     rp, col, val = packed["row_ptr"], packed["col"], packed["val"]
     for n in range(N):
         for e in range(rp[n], rp[n + 1]):
             c = int(col[e])
             nib = (int(val[e >> 1]) >> ((e & 1) * 4)) & 0xF
-            key = ((n // 16) * G + c // 128) * 2 + (c % 32) // 16
-            buckets[key].append(_fragment_byte(n % 16, c % 128) | (nib << 11))
+            key = (n // 16) * G + c // 128
+            buckets[key].append(_fragment_byte(n % 16, c % 128) | (nib << 12))
     ptr = np.zeros(keys + 1, np.int64)
     for k in range(keys):
         ptr[k + 1] = ptr[k] + len(buckets[k])
@@ -157,10 +157,10 @@ def test_tile_lists_regroup_the_csr(N, K, rho, blocks):
 
 
 def test_fragment_byte_covers_each_k_step_once():
-    # every (row, column) of a half-group's four k-steps lands on its own byte
-    # pair, and the sixteen rows x sixteen columns of one k-step fill its 512
-    # bytes exactly
-    for h in (0, 1):
-        cols = [c for c in range(128) if (c % 32) // 16 == h]
-        seen = {_fragment_byte(r, c) for r in range(16) for c in cols}
-        assert len(seen) == 16 * len(cols) and seen == set(range(0, 2048, 2))
+    # every (row, column) of a group lands on its own byte pair, and the
+    # sixteen rows x sixteen columns of one k-step fill its 512 bytes exactly
+    seen = {_fragment_byte(r, c) for r in range(16) for c in range(128)}
+    assert seen == set(range(0, 4096, 2))
+    for s in range(8):
+        cols = [c for c in range(128) if (c % 32) // 4 == s]
+        assert {_fragment_byte(r, c) for r in range(16) for c in cols} == set(range(512 * s, 512 * s + 512, 2))
