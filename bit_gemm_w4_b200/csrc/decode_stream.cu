@@ -159,11 +159,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_stream_kernel(const __grid
     }
     const uint32_t *qbase = p.qweight + warp * 16 + 4 * t;
     uint8_t *ring = smem + L.ring + threadIdx.x * 16;
-    // item (group j of this warp, tile k) into ring slot s
-    // (items past the end copy nothing: a source size of 0 writes zeros, and
-    // the address stays in bounds)
+    // item (group j of this warp, tile k) into the slot at dst (a copy that
+    // is not live writes zeros: a source size of 0; the address stays in
+    // bounds)
     auto issue = [&](int j, int k, uint8_t *dst) {
-        const bool live = j < gpw && (k + 1 < NT || full);
+        // past the warp's last group the copy repeats that group (clamped
+        // below: an L2 hit, never consumed), so only a warp without groups
+        // and a CTA's missing last tile copy nothing
+        const bool live = gpw > 0 && (k + 1 < NT || full);
         const uint32_t *src = qbase + min(j, gpw - 1) * (kWarps * 16);
         cp_async16_if(dst, src + off0[k], live);
         cp_async16_if(dst + kThreads * 16, src + off1[k], live);

@@ -172,11 +172,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tall_kernel(const __grid_c
     const uint32_t wrow = static_cast<uint32_t>(K / 8);
     const uint32_t *qbase = p.qweight + gl * 16 + 4 * t;
     uint8_t *const ring = smem + L.ring + threadIdx.x * 16;
-    // item (group j of this warp, tile k) into the slot at dst (items past the
-    // end copy nothing: a source size of 0 writes zeros, and the address stays
-    // in bounds)
+    // item (group j of this warp, tile k) into the slot at dst (a copy that
+    // is not live writes zeros: a source size of 0; the address stays in
+    // bounds)
     auto issue = [&](int j, int k, uint8_t *dst) {
-        const bool live = j < gpw && k < nv;
+        // past the warp's last group the copy repeats that group (clamped
+        // below: an L2 hit, never consumed)
+        const bool live = gpw > 0 && k < nv;
         const uint32_t *src = qbase + min(j, max(gpw - 1, 0)) * (GL * 16);
         const uint32_t o0 = static_cast<uint32_t>(min(row0 + 16 * k, N - 1)) * wrow;
         const uint32_t o1 = static_cast<uint32_t>(min(row0 + 16 * k + 8, N - 1)) * wrow;
