@@ -75,7 +75,7 @@ DECODE_TRAFFIC = {(4096, 4096): 9.193728e6, (11008, 4096): 24.641024e6,
 # DRAM bytes (read + write) of one launch of the tall-layer decode kernel on
 # the 70B MLP shape (M = 16, density 1 %), from one ncu capture
 # (profiles/decode_tall_kernel_70b_m16.txt). None when the kernel changes.
-TALL_TRAFFIC = 131.396864e6 + 6.799616e6
+TALL_TRAFFIC = 130.875648e6 + 3.997696e6
 
 
 def alg_flops(M: int, N: int, K: int, nnz: int) -> int:

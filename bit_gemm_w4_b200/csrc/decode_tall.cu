@@ -69,7 +69,7 @@ struct TallParams {
     const __nv_bfloat16 *X;   // [M][K]
     __nv_bfloat16 *Y;         // [M][N]
     float *Yf;                // fp32 dense-only output (unfused path) or null
-    const int32_t *tl_ptr;    // residual lists per (tile, group, half-group)
+    const int32_t *tl_ptr;    // residual lists per (16-row tile, group)
     const uint16_t *tl_ent;
     const uint16_t *rscale;
     int M, N, K, G, Gp;
