@@ -1,5 +1,6 @@
-// Streaming decode kernel: Y[M][N] = X[M][K] * W_hat^T for M <= 8, one
-// fused pass over the packed weight.
+// Streaming decode kernel: Y[M][N] = X[M][K] * W_hat^T for M <= 16 where X
+// fits its shared memory, one fused pass over the packed weight (at 9-16
+// tokens two 8-token MMA column tiles share each converted code fragment).
 //
 // MosaicQuant "Methodology" 3. (ZipperEngine): the sparse residual is
 // computed inside the dense 4-bit GEMM pass over the same activations, and

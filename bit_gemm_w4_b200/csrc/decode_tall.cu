@@ -15,13 +15,17 @@
 //     in the streaming kernel, so a group's X fragment is used by one warp
 //     only. That warp loads it straight from L2 (16-byte loads of 64
 //     contiguous bytes per lane and token) at the start of the group and
-//     keeps it in registers across the NT tiles.
+//     keeps it in registers across the tiles. At 9-16 tokens two sets of four
+//     warps split the CTA's tiles and each warp takes every fourth group:
+//     eight accumulator registers per tile and 8-token column tile would not
+//     fit beside the 32-register X fragment otherwise.
 //   * The packed codes stream through a per-thread cp.async ring of R items
 //     (R = 4 or 8, an item being one tile of one group), refilled as soon as
 //     an item is consumed; the slot of item (group j, tile k) is
-//     (j * NT + k) mod R, found at run time once per group, and the item
-//     refilled into it, R items later, has a tile index known at compile
-//     time. No barrier between threads.
+//     (j * NTW + k) mod R (NTW: the warp's tiles), found at run time once per
+//     group, and the item refilled into it, R items later, has a tile index
+//     known at compile time. Items run in pairs after one wait. No barrier
+//     between threads.
 //   * Dense part, per item: exact bf16 codes q - z (a mask into the mantissa
 //     of 128.0, then a subtraction of 128 + z), mma.sync m16n8k16 in fp32 for
 //     one or two 8-token column tiles, the group partial scaled by s in fp32.
@@ -31,12 +35,12 @@
 //     lanes scatter an item's entries as exact bf16 codes into eight zeroed
 //     512-byte fragment tiles, and each k-step that received an entry costs
 //     one more mma.sync per token tile on the X fragment already in
-//     registers; the sums are scaled by the row's
-//     s_r and added in. The residual runs after the group's dense items, in
-//     a loop over the tiles that is not unrolled (the unrolled form outgrew
-//     the instruction cache).
-//   * Reduction-add: the eight warps' partials meet in shared memory in a
-//     fixed order (two stages of four) and are stored once as bf16.
+//     registers; the sums are scaled by the row's s_r and added in. The
+//     residual runs after the group's dense items, in a loop over the tiles
+//     that is not unrolled (the unrolled form outgrew the instruction cache).
+//   * Reduction-add: each warp writes its tiles' sums into its group lane's
+//     slot in shared memory; the slots are summed in a fixed order and the
+//     result is stored once as bf16.
 // The k order inside a group is the packed codes' nibble interleave: k-step s
 // of thread (g, t) covers columns 32t + 4s + {0,1} and 32t + 4s + {2,3}, so
 // thread t's X fragment of a group is columns 32t .. 32t + 31 of its tokens.

@@ -114,11 +114,12 @@ struct L2Prefetch {
 mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaStream_t stream,
                         float *partial = nullptr, const L2Prefetch &pf = L2Prefetch());
 
-// Streaming decode kernel (decode_stream.cu) for M <= 8: persistent, one
+// Streaming decode kernel (decode_stream.cu) for M <= 16: persistent, one
 // CTA per SM over contiguous 16-row tiles, a per-thread cp.async prefetch
 // ring. `partial` and `pf` as for launch_decode. Returns
 // MQ_ERR_UNSUPPORTED (without setting an error message) when X does not fit
-// its shared memory; the caller then takes the register kernel.
+// its shared memory, or when it would leave one CTA per SM over more than
+// one wave; the caller then takes the tall-layer or register kernel.
 mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y,
                                cudaStream_t stream, float *partial = nullptr,
                                const L2Prefetch &pf = L2Prefetch());
