@@ -705,9 +705,18 @@ mq_status mq_linear_path(const mq_weight *w, const void *X, int64_t M, void *Y, 
         return launch_prefill(w, X, M, Y, s);
     }
     switch (path) {
-        case MQ_PATH_DECODE:
-            if (M > 16) return fail(MQ_ERR_UNSUPPORTED, "the decode kernel serves M <= 16");
-            return launch_decode(w, X, static_cast<int>(M), Y, s);
+        case MQ_PATH_DECODE: {
+            // more than 16 tokens: consecutive 16-token slices of X and Y, one
+            // decode launch each (each reads the weight again)
+            const uint16_t *x = static_cast<const uint16_t *>(X);
+            uint16_t *y = static_cast<uint16_t *>(Y);
+            for (int64_t m0 = 0; m0 < M; m0 += 16) {
+                const int mm = static_cast<int>(std::min<int64_t>(16, M - m0));
+                const mq_status st = launch_decode(w, x + m0 * w->d.K, mm, y + m0 * w->d.N, s);
+                if (st) return st;
+            }
+            return MQ_OK;
+        }
         case MQ_PATH_PREFILL:
             return launch_prefill(w, X, M, Y, s);
         default:

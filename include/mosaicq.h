@@ -60,7 +60,7 @@ typedef enum {
  * DECODE for M <= 16, PREFILL otherwise. */
 typedef enum {
     MQ_PATH_AUTO = 0,
-    MQ_PATH_DECODE = 1,  /* register dequant + mma.sync, fused CSR walk; M <= 16 */
+    MQ_PATH_DECODE = 1,  /* the decode kernels (mma.sync); M > 16 in 16-token slices */
     MQ_PATH_PREFILL = 2  /* tcgen05 / TMEM / TMA tensor-core kernel; any M >= 1 */
 } mq_path;
 
@@ -163,8 +163,10 @@ mq_status mq_linear_prefetch(const mq_weight *w, const void *X_dev, int64_t M, v
 
 /* As mq_linear with an explicit kernel choice (mq_linear: the decode
  * kernels for M <= 16 unless X's slice of a very long K exceeds their shared
- * memory, the prefill kernel otherwise). UNSUPPORTED for
- * MQ_PATH_DECODE with M > 16. */
+ * memory, the prefill kernel otherwise). MQ_PATH_DECODE with M > 16 runs
+ * consecutive 16-token slices of X and Y, one decode launch each (the weight
+ * is read once per slice); UNSUPPORTED when the decode kernels cannot take
+ * a slice. */
 mq_status mq_linear_path(const mq_weight *w, const void *X_dev, int64_t M,
                          void *Y_dev, mq_stream stream, mq_path path);
 

@@ -139,9 +139,6 @@ def test_argument_errors(mq, cuda):
     with pytest.raises(mq.MQError) as e:
         w.linear_raw(X.data_ptr(), -1, Y.data_ptr())
     assert e.value.status == mq.INVALID_ARG
-    with pytest.raises(mq.MQError) as e:
-        w.linear_raw(X.data_ptr(), 17, Y.data_ptr(), path="decode")  # decode serves M <= 16
-    assert e.value.status == mq.UNSUPPORTED
     with pytest.raises(mq.MQError):
         w.linear_raw(0, 2, Y.data_ptr())
     small = torch.zeros(4, dtype=torch.float32, device=cuda)
@@ -415,6 +412,17 @@ def test_tall_kernel_sampled_rows(mq, cuda, rho):
         assert r["ok"], (M, r)
         r = oracle_check(Yu[:, rows], X, d)
         assert r["ok"], (M, "unfused", r)
+
+
+@pytest.mark.parametrize("M", [17, 40, 64])
+def test_decode_token_slices(mq, cuda, M):
+    # the decode path past 16 tokens: 16-token slices of X and Y, each a
+    # decode launch (ragged rows, a last slice shorter than 16)
+    W = synth.weight(1000, 1024, std=0.02, outlier_frac=0.01, seed=M + 5)
+    X = synth.activations(M, 1024, seed=M + 6, channels=4, mult=20.0)
+    w, Y = _run(mq, W, X, 0.02, path="decode")
+    r = oracle_check(Y, X, oracle.decompose(W, 0.02))
+    assert r["ok"], r
 
 
 @pytest.mark.parametrize("M", [17, 40])
