@@ -683,6 +683,41 @@ mq_status mq_device_error(const mq_weight *w, mq_stream stream, int32_t *code) {
     return v ? fail(MQ_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait") : MQ_OK;
 }
 
+namespace {
+
+// Y = X * W^T over consecutive 16-token slices, one decode launch each.
+mq_status decode_slices(const mq_weight *w, const void *X, int64_t M, void *Y, cudaStream_t s) {
+    const uint16_t *x = static_cast<const uint16_t *>(X);
+    uint16_t *y = static_cast<uint16_t *>(Y);
+    for (int64_t m0 = 0; m0 < M; m0 += 16) {
+        const int mm = static_cast<int>(std::min<int64_t>(16, M - m0));
+        const mq_status st = launch_decode(w, x + m0 * w->d.K, mm, y + m0 * w->d.N, s);
+        if (st) return st;
+    }
+    return MQ_OK;
+}
+
+// For 17..64 tokens: whether 16-token decode slices beat the prefill kernel,
+// whose one 128-token tile then leaves most SMs idle on short layers. Both
+// sides are estimates fitted to measurements on B200 (the 7B and 70B shapes
+// at 32 and 64 tokens, where they pick the faster side in every case): a
+// 16-token decode launch reads the packed weight at about 0.8 TB/s (1.33 TB/s
+// on layers the tall-layer kernel takes: at least eight 16-row tiles per SM);
+// the prefill kernel spends about 12.8 ns per K column for each wave of
+// 128-row tiles over the SMs.
+bool slices_beat_prefill(const mq_weight *w, int64_t M) {
+    const DeviceWeight &d = w->d;
+    const int64_t sms = sm_count();
+    const double bytes = 0.5 * d.N * d.K + 4.0 * d.N * d.G + 2.5 * d.nnz;
+    const bool tall = (d.N + 15) / 16 >= 8 * sms;
+    const double t_slice = bytes / (tall ? 1.33e12 : 0.8e12);
+    const int64_t waves = ((d.N + 127) / 128 + sms - 1) / sms;
+    const double t_prefill = static_cast<double>(waves) * d.K * 12.8e-9;
+    return static_cast<double>((M + 15) / 16) * t_slice < t_prefill;
+}
+
+}  // namespace
+
 mq_status mq_linear_path(const mq_weight *w, const void *X, int64_t M, void *Y, mq_stream stream,
                          mq_path path) {
     if (!w) return fail(MQ_ERR_INVALID_ARG, "weight handle is NULL");
@@ -701,22 +736,19 @@ mq_status mq_linear_path(const mq_weight *w, const void *X, int64_t M, void *Y, 
             // the decode kernels, unless X's slice cannot fit them (very long K)
             const mq_status st = launch_decode(w, X, static_cast<int>(M), Y, s);
             if (st != MQ_ERR_UNSUPPORTED) return st;
+        } else if (M <= 64 && slices_beat_prefill(w, M)) {
+            // a slice the decode kernels cannot take: the prefill kernel then
+            // computes every row (it rewrites any slice already done)
+            const mq_status st = decode_slices(w, X, M, Y, s);
+            if (st != MQ_ERR_UNSUPPORTED) return st;
         }
         return launch_prefill(w, X, M, Y, s);
     }
     switch (path) {
-        case MQ_PATH_DECODE: {
+        case MQ_PATH_DECODE:
             // more than 16 tokens: consecutive 16-token slices of X and Y, one
             // decode launch each (each reads the weight again)
-            const uint16_t *x = static_cast<const uint16_t *>(X);
-            uint16_t *y = static_cast<uint16_t *>(Y);
-            for (int64_t m0 = 0; m0 < M; m0 += 16) {
-                const int mm = static_cast<int>(std::min<int64_t>(16, M - m0));
-                const mq_status st = launch_decode(w, x + m0 * w->d.K, mm, y + m0 * w->d.N, s);
-                if (st) return st;
-            }
-            return MQ_OK;
-        }
+            return decode_slices(w, X, M, Y, s);
         case MQ_PATH_PREFILL:
             return launch_prefill(w, X, M, Y, s);
         default:

@@ -57,7 +57,9 @@ typedef enum {
 } mq_status;
 
 /* Which kernel mq_linear_path runs. MQ_PATH_AUTO is what mq_linear does:
- * DECODE for M <= 16, PREFILL otherwise. */
+ * DECODE for M <= 16; for 17 <= M <= 64 DECODE (16-token slices) where an
+ * estimate of both sides' times, fitted to B200 measurements, favours it,
+ * else PREFILL; PREFILL for M > 64. */
 typedef enum {
     MQ_PATH_AUTO = 0,
     MQ_PATH_DECODE = 1,  /* the decode kernels (mma.sync); M > 16 in 16-token slices */
@@ -163,7 +165,8 @@ mq_status mq_linear_prefetch(const mq_weight *w, const void *X_dev, int64_t M, v
 
 /* As mq_linear with an explicit kernel choice (mq_linear: the decode
  * kernels for M <= 16 unless X's slice of a very long K exceeds their shared
- * memory, the prefill kernel otherwise). MQ_PATH_DECODE with M > 16 runs
+ * memory, 16-token decode slices or the prefill kernel for 17..64 tokens as
+ * MQ_PATH_AUTO describes, the prefill kernel above). MQ_PATH_DECODE with M > 16 runs
  * consecutive 16-token slices of X and Y, one decode launch each (the weight
  * is read once per slice); UNSUPPORTED when the decode kernels cannot take
  * a slice. */

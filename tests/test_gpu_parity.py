@@ -62,7 +62,7 @@ def test_decode_token_counts_ragged_rows(mq, cuda, M):
 def test_prefill_token_counts(mq, cuda, M):
     W = synth.weight(136, 512, std=0.02, outlier_frac=0.01, seed=M)
     X = synth.activations(M, 512, seed=200 + M, channels=8, mult=30.0)
-    w, Y = _run(mq, W, X, 0.01, path="auto")
+    w, Y = _run(mq, W, X, 0.01, path="prefill")
     r = oracle_check(Y, X, oracle.decompose(W, 0.01))
     assert r["ok"], r
 
@@ -425,6 +425,27 @@ def test_decode_token_slices(mq, cuda, M):
     assert r["ok"], r
 
 
+@pytest.mark.parametrize("M", [17, 40, 64])
+def test_auto_token_counts_17_to_64(mq, cuda, M):
+    # mq_linear at 17-64 tokens: decode slices on a short layer (the
+    # estimate favours them), the prefill kernel on an 11008 x 4096 layer at
+    # 32 or more tokens (it favours prefill there), checked on sampled rows
+    W = synth.weight(136, 512, std=0.02, outlier_frac=0.01, seed=M + 40)
+    X = synth.activations(M, 512, seed=M + 41, channels=8, mult=30.0)
+    w, Y = _run(mq, W, X, 0.01)
+    r = oracle_check(Y, X, oracle.decompose(W, 0.01))
+    assert r["ok"], r
+    if M >= 32:
+        N, K = 11008, 4096
+        W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=M + 42)
+        X = synth.activations(M, K, seed=M + 43, channels=4, mult=20.0)
+        w, Y = _run(mq, W, X, 0.005)
+        rows = np.unique(np.concatenate([np.arange(0, 24), np.arange(N - 24, N),
+                                         np.random.default_rng(M).choice(N, 48, replace=False)]))
+        r = oracle_check(Y[:, rows], X, oracle.decompose(np.ascontiguousarray(W[rows]), 0.005))
+        assert r["ok"], r
+
+
 @pytest.mark.parametrize("M", [17, 40])
 def test_longest_k_prefill(mq, cuda, M):
     # K = 65536 at more than 16 tokens: the prefill kernel reads 512 scale
@@ -432,7 +453,7 @@ def test_longest_k_prefill(mq, cuda, M):
     N, K = 160, 65536
     W = synth.weight(N, K, std=0.02, outlier_frac=0.005, seed=96)
     X = synth.activations(M, K, seed=97, channels=4, mult=20.0)
-    w, Y = _run(mq, W, X, 0.002)
+    w, Y = _run(mq, W, X, 0.002, path="prefill")
     r = oracle_check(Y, X, oracle.decompose(W, 0.002))
     assert r["ok"], r
 
