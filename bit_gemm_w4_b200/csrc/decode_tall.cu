@@ -1,6 +1,6 @@
 // Tall-layer decode kernel: Y[M][N] = X[M][K] * W_hat^T for 2 <= M <= 16 on
-// layers tall enough to give every CTA four or more 16-row tiles at two CTAs
-// per SM (a 70B MLP projection, 28672 x 8192), one fused pass.
+// layers tall enough to give every CTA two or more 16-row tiles at two CTAs
+// per SM (a 70B MLP projection, 28672 x 8192: six or seven), one fused pass.
 //
 // MosaicQuant "Methodology" 3. (ZipperEngine): the sparse residual is
 // computed inside the dense 4-bit GEMM pass over the same activations, and
@@ -10,7 +10,7 @@
 // At 16 tokens and K = 8192 X alone is 256 KB, more than an SM holds, and
 // even at 2-8 tokens it leaves one CTA per SM for grids of two waves. Here
 // nothing of X is staged:
-//   * Persistent grid of two CTAs per SM (NT = 4..8 contiguous 16-row tiles
+//   * Persistent grid of two CTAs per SM (NT = 2..8 contiguous 16-row tiles
 //     each); warp w takes groups w, w + 8, ... of every tile of its CTA, as
 //     in the streaming kernel, so a group's X fragment is used by one warp
 //     only. That warp loads it straight from L2 (16-byte loads of 64
@@ -60,7 +60,7 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kTMin = 4;                   // fewest tiles per CTA (X is read once per CTA and group)
+constexpr int kTMin = 2;                   // fewest tiles per CTA (X is read once per CTA and group)
 constexpr int kTMax = 8;                   // most tiles per CTA (one accumulator set each)
 constexpr int kSlotBytes = 2 * kThreads * 16;  // one item: 16 bytes of rows g and g + 8 per thread
 constexpr int kFragBytes = 8 * 512;        // per warp: the A fragments of a group's eight k-steps
@@ -413,6 +413,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tall_kernel(const __grid_c
 template <int MX, int R>
 void *kernel_for(int nt) {
     switch (nt) {
+        case 2: return reinterpret_cast<void *>(decode_tall_kernel<MX, 2, R>);
+        case 3: return reinterpret_cast<void *>(decode_tall_kernel<MX, 3, R>);
         case 4: return reinterpret_cast<void *>(decode_tall_kernel<MX, 4, R>);
         case 5: return reinterpret_cast<void *>(decode_tall_kernel<MX, 5, R>);
         case 6: return reinterpret_cast<void *>(decode_tall_kernel<MX, 6, R>);

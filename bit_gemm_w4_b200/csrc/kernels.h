@@ -125,7 +125,7 @@ mq_status launch_decode_stream(const mq_weight *w, const void *X, int M, void *Y
                                const L2Prefetch &pf = L2Prefetch());
 
 // Tall-layer decode kernel (decode_tall.cu) for 2 <= M <= 16 on layers of
-// at least four 16-row tiles per CTA at two CTAs per SM: X from L2, a
+// at least two 16-row tiles per CTA at two CTAs per SM: X from L2, a
 // per-thread item ring, the residual as tensor-core k-steps from the
 // per-tile lists (DeviceWeight::tl_ptr). `partial` and `pf` as for
 // launch_decode. Returns MQ_ERR_UNSUPPORTED (without setting an error
