@@ -469,6 +469,8 @@ mq_status launch_decode(const mq_weight *w, const void *X, int M, void *Y, cudaS
         if (st != MQ_ERR_UNSUPPORTED) return st;
     }
     if (M > 8) {
+        // 9-16 tokens on tall layers the tall-layer kernel declined (a CTA's
+        // residual lists beyond their shared-memory budget)
         const mq_status st = launch_decode_wide(w, X, M, Y, stream, partial, pf);
         if (st != MQ_ERR_UNSUPPORTED) return st;
     }
