@@ -146,6 +146,8 @@ def _tile_expected(N, K, packed):
     (300, 640, 0.05, None),      # ragged last tile, five groups
     (256, 1024, 0.0, 0.25),      # block mode
     (128, 256, 0.0, None),       # no residual
+    (17, 128, 0.3, None),        # one group, a second tile of one row
+    (1, 256, 0.5, None),         # one row: half its entries in the residual
 ])
 def test_tile_lists_regroup_the_csr(N, K, rho, blocks):
     W = synth.weight(N, K, std=0.02, outlier_frac=0.01, seed=3 * N + K)
