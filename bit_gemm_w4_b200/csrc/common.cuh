@@ -123,16 +123,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
-// 1D bulk copy global -> shared (16-byte aligned addresses, size % 16 == 0).
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
-                                          uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-            "r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -245,12 +235,6 @@ __device__ __forceinline__ int col_lower_bound(const uint16_t *colp, int coff, i
 
 
 // ---------------------------------------------------------------- math
-// bf16x2 (128 + q_lo, 128 + q_hi) for the nibble pair at bits [0,4) and
-// [16,20) of w: the codes become the low mantissa bits of 128.0 exactly.
-__device__ __forceinline__ uint32_t nib_pair_bias128(uint32_t w) {
-    return (w & 0x000F000Fu) | 0x43004300u;
-}
-
 // The bias words of the code conversions, bf16x2 (128, 128) and the int8
 // sign-bias bytes. Kernels take them as launch parameters: held in a
 // register, (w & mask) | bias is one LOP3, where a second 32-bit immediate
@@ -266,8 +250,9 @@ __device__ __forceinline__ uint32_t mask_or(uint32_t w, uint32_t bias) {
 }
 
 // Four int8 bytes q - z from the low nibble of each byte of w, with the
-// sign-bias word in a register (kBiasI8): the same arithmetic as
-// codes_minus_zero in two LOP3s and one add.
+// sign-bias word in a register (kBiasI8): (nibble | 0x80) - z never borrows
+// across bytes (z <= 15), and ^ 0x80 restores the sign; two LOP3s and one
+// add.
 __device__ __forceinline__ uint32_t codes_minus_zero_r(uint32_t w, uint32_t zz4, uint32_t bias8) {
     return (mask_or<0x0F0F0F0Fu>(w, bias8) - zz4) ^ bias8;
 }
@@ -297,12 +282,6 @@ __device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4]
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Four int8 bytes q - z from four nibbles 0..15 held in the low half of each
-// byte of v: (v | 0x80) - z never borrows across bytes; ^ 0x80 restores sign.
-__device__ __forceinline__ uint32_t codes_minus_zero(uint32_t nib4, uint32_t zz4) {
-    return ((nib4 | 0x80808080u) - zz4) ^ 0x80808080u;
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) {
